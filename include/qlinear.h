@@ -1,0 +1,181 @@
+/*
+ * qlinear.h -- C ABI of the weight-only-quantized linear layer for NVIDIA B200 (sm_100a).
+ *
+ *   y[M, N] = x[M, K] . dequant(Wq)[K, N],   M = 1..16 activation rows (LLM decoding)
+ *
+ * Formats
+ *   W2 / W4 / W8 : group-wise asymmetric uniform codes, one fp16 scale s and one
+ *                  fp16 zero z (an integer) per 128-element group along K per
+ *                  column; w = s * (q - z).  Sources: QFactory (ATC'25) page,
+ *                  "问题与动机" and observation 1 (fine-grained asymmetric group-wise
+ *                  quantization, group size 128, W8/W4/W2).
+ *   LUT4         : 4-bit indices into a 16-entry fp16 table with an fp32 absmax per
+ *                  64-element block along K per column; w = lut[q] * absmax.
+ *                  Source: "Fast NF4 Dequantization Kernels for Large Language Model
+ *                  Inference" page, abstract and method section (NF4 lookup table).
+ *   W4 + outliers: W4 dense part plus fp16 outliers in Tile-COO (128 x 128 K x N
+ *                  tiles, uint32 per-tile offsets, uint8 in-tile (row, col) pairs);
+ *                  y = x . dequant(W_dense) + x . W_outlier.  Source: FlashQuant page,
+ *                  English abstract (fused dense GEMM + sparse outlier path, sparse-
+ *                  dense tiling, Tile-COO encoding).
+ *
+ * Every GEMV uses the deferred-dequantization identity of the QFactory page
+ * (observation 2, J-matrix expansion, Table 2) in its weight-only form:
+ *   y[m, n] = sum_g s[g, n] * ( sum_{k in g} q[k, n] x[m, k] - z[g, n] * sum_{k in g} x[m, k] ).
+ *
+ * Conventions (all entry points)
+ *   - fp16 arguments are IEEE binary16 bit patterns (uint16_t); fp32 are IEEE binary32.
+ *   - "device" pointers point to memory of the current CUDA device, owned by the caller;
+ *     the library never allocates, frees or synchronizes.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream); device work is enqueued
+ *     asynchronously on it and the call returns without waiting.
+ *   - The return value is a ql_status.  Argument errors are detected on the host before
+ *     anything is enqueued; QL_ERR_CUDA reports a launch failure (cudaGetLastError).
+ *   - Shapes: K % 128 == 0, N % 16 == 0, 1 <= M <= 16; the outlier variant also needs
+ *     N % 128 == 0.  All 2-bit shapes with K % 128 == 0 are accepted.
+ *   - Calls are thread-safe; two calls that share one workspace must not overlap in time
+ *     (issue them on one stream).
+ *
+ * Canonical (packer input) layouts, host memory:
+ *   uniform codes : uint32[K / P][N], P = 32 / bits; word (j, n) bits [bits*i, bits*i + bits)
+ *                   hold the code of weight (P*j + i, n)
+ *   scales, zeros : fp16 [K / 128][N]
+ *   LUT4 codes    : uint8 [K / 2][N]; low nibble = even k, high nibble = odd k
+ *   LUT4 absmax   : fp32 [K / 64][N];  lut: fp16 [16]
+ *   Tile-COO      : tiles t = kt * (N / 128) + nt; offsets uint32[T + 1] (offsets[0] = 0,
+ *                   offsets[T] = nnz); rc uint8[nnz][2] = (k - 128 kt, n - 128 nt);
+ *                   vals fp16[nnz].  The kernels read this layout directly.
+ */
+#ifndef QLINEAR_H_
+#define QLINEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QL_OK = 0,
+  QL_ERR_NULL = 1,        /* a required pointer is NULL */
+  QL_ERR_SHAPE = 2,       /* M, N, K, group or block outside the supported set */
+  QL_ERR_ALIGN = 3,       /* a pointer is not aligned as documented */
+  QL_ERR_UNSUPPORTED = 4, /* unknown format */
+  QL_ERR_WORKSPACE = 5,   /* workspace missing or smaller than qlinear_workspace_bytes() */
+  QL_ERR_CUDA = 6         /* a CUDA runtime call or kernel launch failed */
+} ql_status;
+
+typedef enum { QL_FMT_W2 = 2, QL_FMT_W4 = 4, QL_FMT_W8 = 8, QL_FMT_LUT4 = 16 } ql_format;
+
+/* Opaque stream handle, ABI-compatible with cudaStream_t. */
+typedef struct CUstream_st* ql_stream_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* ql_status_str(int status);
+
+/* ---------------------------------------------------------------------------
+ * Host-side packer.  Host pointers, caller-allocated outputs, no device work.
+ * The packed codes have exactly the byte count of the canonical codes; the packed
+ * quantization parameters have exactly the byte count of the canonical ones.
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of packed codes (= canonical code bytes, K * N * bits / 8); 0 on a bad shape. */
+size_t qlinear_packed_bytes(int fmt, int N, int K);
+
+/* Bytes of packed parameters: scales or zeros (fp16, K/128 * N each) for W2/W4/W8,
+ * absmax (fp32, K/64 * N) for LUT4; 0 on a bad shape. */
+size_t qlinear_params_bytes(int fmt, int N, int K);
+
+/* Reorder canonical codes into the kernel layout (a bijection on code fields):
+ * each warp of the GEMV then issues one 128/256-bit coalesced load per 16-column
+ * tile and 128-element group, and each code lands where the tensor-core fragment
+ * wants it.  `canonical` and `packed` are host buffers of qlinear_packed_bytes(). */
+ql_status qlinear_pack(int fmt, const void* canonical, void* packed, int N, int K);
+
+/* Reorder one canonical parameter array into the kernel layout: call it for the
+ * scales and again for the zeros of W2/W4/W8 (fp16 [K/128][N]), or for the absmax of
+ * LUT4 (fp32 [K/64][N]).  Host buffers of qlinear_params_bytes(). */
+ql_status qlinear_pack_params(int fmt, const void* canonical, void* packed, int N, int K);
+
+/* ---------------------------------------------------------------------------
+ * Workspace.  The split-K fix-up needs fp32 partial sums and per-tile arrival
+ * counters.  The caller allocates qlinear_workspace_bytes() on the device (256-byte
+ * aligned) and zero-fills it ONCE before its first use; every completed call leaves
+ * the counters at zero again, so no per-call clearing is needed.
+ * ------------------------------------------------------------------------- */
+
+/* Workspace bytes for a call with these arguments on the current device; 0 if none. */
+size_t qlinear_workspace_bytes(int fmt, int M, int N, int K);
+
+/* ---------------------------------------------------------------------------
+ * Hot path (device pointers, asynchronous on `stream`).
+ *   x       : fp16 [M][K] row-major, 16-byte aligned
+ *   qweight : packed codes from qlinear_pack, 32-byte aligned
+ *   scales, zeros : packed fp16 parameters from qlinear_pack_params, 4-byte aligned
+ *   y       : fp16 [M][N] row-major output (round-to-nearest-even of an fp32 sum)
+ *   group   : must be 128
+ * ------------------------------------------------------------------------- */
+
+ql_status qlinear_w4a16(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                        const uint16_t* zeros, uint16_t* y, int M, int N, int K, int group,
+                        void* workspace, size_t workspace_bytes, ql_stream_t stream);
+
+ql_status qlinear_w2a16(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                        const uint16_t* zeros, uint16_t* y, int M, int N, int K, int group,
+                        void* workspace, size_t workspace_bytes, ql_stream_t stream);
+
+ql_status qlinear_w8a16(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                        const uint16_t* zeros, uint16_t* y, int M, int N, int K, int group,
+                        void* workspace, size_t workspace_bytes, ql_stream_t stream);
+
+/* LUT4: codes packed by qlinear_pack(QL_FMT_LUT4), 32-byte aligned; lut16: fp16[16]
+ * (device); absmax packed by qlinear_pack_params(QL_FMT_LUT4), 16-byte aligned;
+ * block must be 64. */
+ql_status qlinear_lut4(const uint16_t* x, const uint8_t* codes, const uint16_t* lut16,
+                       const float* absmax, uint16_t* y, int M, int N, int K, int block,
+                       void* workspace, size_t workspace_bytes, ql_stream_t stream);
+
+/* W4 dense part (as qlinear_w4a16) plus the canonical Tile-COO outliers, processed in
+ * the same kernel: tile_offsets uint32[T+1] (4-byte aligned), tile_rc uint8[nnz][2]
+ * (2-byte aligned), tile_vals fp16[nnz] (2-byte aligned), T = (K/128) * (N/128).
+ * The dense code of every outlier position must equal its group's zero code. */
+ql_status qlinear_w4a16_outlier(const uint16_t* x, const uint32_t* qweight,
+                                const uint16_t* scales, const uint16_t* zeros,
+                                const uint32_t* tile_offsets, const uint8_t* tile_rc,
+                                const uint16_t* tile_vals, uint16_t* y, int M, int N, int K,
+                                int group, void* workspace, size_t workspace_bytes,
+                                ql_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Debug entries (device pointers, asynchronous).  They decode the packed layout
+ * with the same fragment-extraction code the GEMV kernels use.
+ *   qlinear_debug_unpack : codes uint8 [K][N] (canonical order, one code per byte)
+ *   qlinear_debug_dequant: w fp32 [K][N]; p0 = packed scales (fp16) or the device
+ *                          lut16 (fp16[16]); p1 = packed zeros (fp16) or packed
+ *                          absmax (fp32).  W2/W4/W8 give s*(q-z) (exact in fp32);
+ *                          LUT4 gives fp32(lut[q]) * absmax rounded to nearest.
+ * ------------------------------------------------------------------------- */
+ql_status qlinear_debug_unpack(int fmt, const void* packed, uint8_t* codes, int N, int K,
+                               ql_stream_t stream);
+ql_status qlinear_debug_dequant(int fmt, const void* packed, const void* p0, const void* p1,
+                                float* w, int N, int K, ql_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Launch plan (host, for tuning and reporting): CTAs, warps per CTA and work units of
+ * the GEMV launch that a call with these arguments would make on the current device.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int ctas;         /* persistent CTAs launched */
+  int warps;        /* warps per CTA */
+  int tiles_per_warp;
+  long long units;  /* (128-column block, 128-element group) work units */
+  int m_bucket;     /* 1: M <= 8, 2: M <= 16 */
+} ql_plan;
+
+ql_status qlinear_plan(int fmt, int M, int N, int K, ql_plan* plan);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLINEAR_H_ */
