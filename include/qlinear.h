@@ -98,6 +98,15 @@ ql_status qlinear_pack(int fmt, const void* canonical, void* packed, int N, int 
  * LUT4 (fp32 [K/64][N]).  Host buffers of qlinear_params_bytes(). */
 ql_status qlinear_pack_params(int fmt, const void* canonical, void* packed, int N, int K);
 
+/* Reorder canonical Tile-COO (tiles numbered t = kt * (N/128) + nt) into the order the
+ * fused outlier kernel walks them, t' = nt * (K/128) + kt, so that the outliers of one run
+ * of (block, group) work units are contiguous.  Entries keep their in-tile order.  Host
+ * buffers: offsets uint32[T+1] in and out, rc uint8[nnz][2], vals fp16[nnz].
+ * Returns QL_ERR_SHAPE for N or K not multiples of 128 or non-monotone offsets. */
+ql_status qlinear_pack_tilecoo(const uint32_t* offsets, const uint8_t* rc, const uint16_t* vals,
+                               int N, int K, uint32_t* offsets_out, uint8_t* rc_out,
+                               uint16_t* vals_out);
+
 /* ---------------------------------------------------------------------------
  * Workspace.  The split-K fix-up needs fp32 partial sums and per-tile arrival
  * counters.  The caller allocates qlinear_workspace_bytes() on the device (256-byte
@@ -136,10 +145,12 @@ ql_status qlinear_lut4(const uint16_t* x, const uint8_t* codes, const uint16_t* 
                        const float* absmax, uint16_t* y, int M, int N, int K, int block,
                        void* workspace, size_t workspace_bytes, ql_stream_t stream);
 
-/* W4 dense part (as qlinear_w4a16) plus the canonical Tile-COO outliers, processed in
- * the same kernel: tile_offsets uint32[T+1] (4-byte aligned), tile_rc uint8[nnz][2]
+/* W4 dense part (as qlinear_w4a16) plus the Tile-COO outliers, processed in the same
+ * kernel.  The Tile-COO arrays are those written by qlinear_pack_tilecoo (tiles in
+ * block-major order): tile_offsets uint32[T+1] (4-byte aligned), tile_rc uint8[nnz][2]
  * (2-byte aligned), tile_vals fp16[nnz] (2-byte aligned), T = (K/128) * (N/128).
- * The dense code of every outlier position must equal its group's zero code. */
+ * Needs N % 128 == 0 and K <= 65536.  The dense code of every outlier position should
+ * hold its group's zero code (then the dense part contributes nothing there). */
 ql_status qlinear_w4a16_outlier(const uint16_t* x, const uint32_t* qweight,
                                 const uint16_t* scales, const uint16_t* zeros,
                                 const uint32_t* tile_offsets, const uint8_t* tile_rc,

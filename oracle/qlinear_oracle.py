@@ -187,13 +187,12 @@ def tilecoo_to_dense(offsets: np.ndarray, rc: np.ndarray, vals: np.ndarray, K: i
         out = np.zeros((K, N), dtype=np.float64)
         np.add.at(out, (k, n), v)
         return out
-    cols = np.asarray(cols)
+    cols = np.asarray(cols, dtype=np.int64)
     out = np.zeros((K, len(cols)), dtype=np.float64)
-    where = {int(c): i for i, c in enumerate(cols)}
-    for kk, nn, vv in zip(k, n, v):
-        i = where.get(int(nn))
-        if i is not None:
-            out[kk, i] += vv
+    pos = np.full(N, -1, dtype=np.int64)
+    pos[cols] = np.arange(len(cols))
+    keep = pos[n] >= 0
+    np.add.at(out, (k[keep], pos[n[keep]]), v[keep])
     return out
 
 

@@ -185,16 +185,17 @@ def lut16(seed: int) -> np.ndarray:
 
 
 def _nearest_lut_codes(r: np.ndarray, lut: np.ndarray) -> np.ndarray:
-    """Index of the nearest table entry for each ratio (fp64), lower index on ties."""
+    """Index of the nearest table entry for each ratio (fp64 distances), lower index on ties.
+
+    The table is sorted, so |r - lut[c]| (fp64) does not increase towards r from either
+    side: the minimum is one of the two entries around r's insertion point.
+    """
     lut64 = lut.astype(np.float64)
-    best = np.zeros(r.shape, dtype=np.uint8)
-    bestd = np.abs(r - lut64[0])
-    for c in range(1, 16):
-        d = np.abs(r - lut64[c])
-        better = d < bestd  # strict: an exact tie keeps the lower index
-        best = np.where(better, np.uint8(c), best)
-        bestd = np.where(better, d, bestd)
-    return best
+    hi = np.clip(np.searchsorted(lut64, r, side="left"), 1, 15)
+    lo = hi - 1
+    dlo = np.abs(r - lut64[lo])
+    dhi = np.abs(r - lut64[hi])
+    return np.where(dlo <= dhi, lo, hi).astype(np.uint8)
 
 
 def lut4_layer(seed: int, K: int, N: int, block: int = LUT_BLOCK,

@@ -1,0 +1,142 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every declared
+symbol, packs on the host, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def ql():
+    import weight_only_quantized_gemv_b200 as q
+    return q
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)
+    return [n for n in names if n not in ("if", "while")]
+
+
+def test_exports_every_declared_symbol(ql):
+    declared = _declared_functions()
+    assert "qlinear_w4a16" in declared and "qlinear_pack" in declared
+    lib = ctypes.CDLL(ql.LIBRARY_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(ql.EXPORTED)
+
+
+def test_status_strings(ql):
+    for s in range(7):
+        assert ql._lib.ql_status_str(s)
+    assert b"unknown" in ql._lib.ql_status_str(99)
+
+
+@pytest.mark.parametrize("fmt,bits", [(2, 2), (4, 4), (8, 8), (16, 4)])
+def test_pack_is_a_permutation_of_code_fields(ql, fmt, bits):
+    K, N = 384, 208  # 13 tiles: one full 128-column block and a ragged one
+    rs = np.random.default_rng(fmt)
+    nbytes = K * N * bits // 8
+    canon = rs.integers(0, 256, size=nbytes, dtype=np.uint8)
+    packed = ql.qlinear_pack(fmt, canon, N, K)
+    assert packed.nbytes == nbytes
+    # multiset of code fields is preserved
+    def fields(a):
+        v = a.view(np.uint8)
+        if bits == 8:
+            return np.bincount(v, minlength=256)
+        if bits == 4:
+            return np.bincount(np.concatenate([v & 15, v >> 4]), minlength=16)
+        return np.bincount(np.concatenate([(v >> s) & 3 for s in (0, 2, 4, 6)]), minlength=4)
+    assert np.array_equal(fields(canon), fields(packed))
+    # a single nonzero code lands in exactly one field
+    one = np.zeros(nbytes, dtype=np.uint8)
+    one[nbytes // 3] = 1
+    p1 = ql.qlinear_pack(fmt, one, N, K)
+    assert int(np.count_nonzero(p1)) == 1
+    # deterministic
+    assert np.array_equal(packed, ql.qlinear_pack(fmt, canon, N, K))
+
+
+def test_pack_params_permutes(ql):
+    K, N = 512, 48
+    a = np.arange((K // 128) * N, dtype=np.float16).reshape(K // 128, N)
+    p = ql.qlinear_pack_params(4, a, N, K)
+    assert sorted(p.reshape(-1).tolist()) == sorted(a.reshape(-1).tolist())
+    b = np.arange((K // 64) * N, dtype=np.float32).reshape(K // 64, N)
+    q = ql.qlinear_pack_params(16, b, N, K)
+    assert sorted(q.reshape(-1).tolist()) == sorted(b.reshape(-1).tolist())
+
+
+def test_pack_tilecoo_reorders_tiles(ql):
+    from synth import gen
+    K, N = 384, 256
+    lay = gen.outlier_layer(4100, K, N)
+    o2, r2, v2 = ql.qlinear_pack_tilecoo(lay.tile_offsets, lay.tile_rc, lay.tile_vals, N, K)
+    NB, KT = N // 128, K // 128
+    for nt in range(NB):
+        for kt in range(KT):
+            t = kt * NB + nt
+            t2 = nt * KT + kt
+            a, b = lay.tile_offsets[t], lay.tile_offsets[t + 1]
+            c, d = o2[t2], o2[t2 + 1]
+            assert b - a == d - c
+            assert np.array_equal(lay.tile_rc[a:b], r2[c:d])
+            assert np.array_equal(lay.tile_vals[a:b].view(np.uint16), v2[c:d].view(np.uint16))
+    bad = lay.tile_offsets.copy()
+    bad[2], bad[3] = bad[3], bad[2] + 1
+    with pytest.raises(ql.QLinearError):
+        ql.qlinear_pack_tilecoo(bad, lay.tile_rc, lay.tile_vals, N, K)
+
+
+def test_packer_rejects_bad_shapes(ql):
+    assert ql.qlinear_packed_bytes(4, 24, 128) == 0
+    assert ql.qlinear_packed_bytes(4, 16, 100) == 0
+    assert ql.qlinear_packed_bytes(3, 16, 128) == 0
+    assert ql.qlinear_packed_bytes(4, 16, 128) == 16 * 128 // 2
+    assert ql._lib.qlinear_pack(4, None, None, 16, 128) == 1
+    buf = np.zeros(64, dtype=np.uint8)
+    assert ql._lib.qlinear_pack(4, buf.ctypes.data, buf.ctypes.data, 24, 128) == 2
+    assert ql._lib.qlinear_pack(5, buf.ctypes.data, buf.ctypes.data, 16, 128) == 4
+
+
+def test_hot_path_validates_before_any_device_work(ql):
+    """Argument errors come back as status codes; no CUDA call is made for them."""
+    lib = ql._lib
+    a = 1 << 20  # an aligned, never-dereferenced address
+    ok = dict(x=a, q=a, s=a, z=a, y=a, M=1, N=128, K=128, g=128, ws=a, wsb=1 << 20, st=None)
+
+    def call(fn=lib.qlinear_w4a16, **kw):
+        d = dict(ok, **kw)
+        return fn(d["x"], d["q"], d["s"], d["z"], d["y"], d["M"], d["N"], d["K"], d["g"], d["ws"],
+                  d["wsb"], d["st"])
+    assert call(x=None) == 1
+    assert call(y=None) == 1
+    assert call(M=0) == 2 and call(M=17) == 2
+    assert call(N=24) == 2 and call(K=100) == 2 and call(g=64) == 2
+    assert call(x=a + 2) == 3 and call(q=a + 16) == 3 and call(s=a + 2) == 3
+    assert call(fn=lib.qlinear_w2a16, K=192) == 2
+    assert call(fn=lib.qlinear_w8a16, N=8) == 2
+    # LUT4 wants block 64
+    assert lib.qlinear_lut4(a, a, a, a, a, 1, 128, 128, 128, a, 1 << 20, None) == 2
+    # outliers need N % 128 == 0
+    assert lib.qlinear_w4a16_outlier(a, a, a, a, a, a, a, a, 1, 144, 128, 128, a, 1 << 20, None) == 2
+    assert lib.qlinear_w4a16_outlier(a, a, a, a, None, a, a, a, 1, 128, 128, 128, a, 1 << 20, None) == 1
+    assert lib.qlinear_debug_unpack(4, None, a, 128, 128, None) == 1
+    assert lib.qlinear_debug_unpack(3, a, a, 128, 128, None) == 4
+    assert lib.qlinear_workspace_bytes(4, 0, 128, 128) == 0
+
+
+def test_graft_entry_build_is_idempotent():
+    import __graft_entry__ as ge
+    ge.build()
+    ge.build()

@@ -1,0 +1,207 @@
+"""Python binding of ``libqlinear.so``: the weight-only-quantized linear layer on B200.
+
+Argument marshalling only.  Every function here forwards to the C entry point of
+the same name in ``include/qlinear.h``; device arguments are ``torch.Tensor``
+objects on the current CUDA device (their ``data_ptr()`` is passed), host
+arguments of the packers are NumPy arrays.  A non-OK status raises
+``QLinearError``.  There is no fallback: if the shared library is missing, the
+import fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_HERE, "libqlinear.so")
+
+if not os.path.exists(LIBRARY_PATH):
+    raise ImportError(
+        f"{LIBRARY_PATH} is missing: build it with "
+        "`python -c 'import __graft_entry__ as g; g.build()'` or "
+        "`python weight_only_quantized_gemv_b200/build.py`")
+
+_lib = ctypes.CDLL(LIBRARY_PATH)
+
+QL_FMT_W2, QL_FMT_W4, QL_FMT_W8, QL_FMT_LUT4 = 2, 4, 8, 16
+FORMATS = {"w2": QL_FMT_W2, "w4": QL_FMT_W4, "w8": QL_FMT_W8, "lut4": QL_FMT_LUT4}
+STATUS = {0: "QL_OK", 1: "QL_ERR_NULL", 2: "QL_ERR_SHAPE", 3: "QL_ERR_ALIGN",
+          4: "QL_ERR_UNSUPPORTED", 5: "QL_ERR_WORKSPACE", 6: "QL_ERR_CUDA"}
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+
+class ql_plan(ctypes.Structure):
+    _fields_ = [("ctas", ctypes.c_int), ("warps", ctypes.c_int), ("tiles_per_warp", ctypes.c_int),
+                ("units", ctypes.c_longlong), ("m_bucket", ctypes.c_int)]
+
+
+_SIGS = {
+    "ql_status_str": (ctypes.c_char_p, [_I]),
+    "qlinear_packed_bytes": (_SZ, [_I, _I, _I]),
+    "qlinear_params_bytes": (_SZ, [_I, _I, _I]),
+    "qlinear_pack": (_I, [_I, _P, _P, _I, _I]),
+    "qlinear_pack_params": (_I, [_I, _P, _P, _I, _I]),
+    "qlinear_pack_tilecoo": (_I, [_P, _P, _P, _I, _I, _P, _P, _P]),
+    "qlinear_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+    "qlinear_w4a16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
+    "qlinear_w2a16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
+    "qlinear_w8a16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
+    "qlinear_lut4": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
+    "qlinear_w4a16_outlier": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
+    "qlinear_debug_unpack": (_I, [_I, _P, _P, _I, _I, _P]),
+    "qlinear_debug_dequant": (_I, [_I, _P, _P, _P, _P, _I, _I, _P]),
+    "qlinear_plan": (_I, [_I, _I, _I, _I, ctypes.POINTER(ql_plan)]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+class QLinearError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = _lib.ql_status_str(status).decode()
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({msg})")
+        self.status = status
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise QLinearError(status, where)
+
+
+def _ptr(t) -> Optional[int]:
+    """Device pointer of a torch tensor, or None."""
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _np_ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+# ---------------------------------------------------------------------------
+# host packer (NumPy in, NumPy out)
+
+
+def qlinear_packed_bytes(fmt: int, N: int, K: int) -> int:
+    return int(_lib.qlinear_packed_bytes(fmt, N, K))
+
+
+def qlinear_params_bytes(fmt: int, N: int, K: int) -> int:
+    return int(_lib.qlinear_params_bytes(fmt, N, K))
+
+
+def qlinear_pack(fmt: int, canonical: np.ndarray, N: int, K: int) -> np.ndarray:
+    canonical = np.ascontiguousarray(canonical)
+    out = np.empty(qlinear_packed_bytes(fmt, N, K), dtype=np.uint8)
+    if out.size != canonical.nbytes:
+        raise QLinearError(2, "qlinear_pack")
+    _check(_lib.qlinear_pack(fmt, _np_ptr(canonical), _np_ptr(out), N, K), "qlinear_pack")
+    return out
+
+
+def qlinear_pack_params(fmt: int, canonical: np.ndarray, N: int, K: int) -> np.ndarray:
+    canonical = np.ascontiguousarray(canonical)
+    out = np.empty(canonical.shape, dtype=canonical.dtype)
+    if canonical.nbytes != qlinear_params_bytes(fmt, N, K):
+        raise QLinearError(2, "qlinear_pack_params")
+    _check(_lib.qlinear_pack_params(fmt, _np_ptr(canonical), _np_ptr(out), N, K),
+           "qlinear_pack_params")
+    return out
+
+
+def qlinear_pack_tilecoo(offsets: np.ndarray, rc: np.ndarray, vals: np.ndarray, N: int, K: int):
+    offsets = np.ascontiguousarray(offsets, dtype=np.uint32)
+    rc = np.ascontiguousarray(rc, dtype=np.uint8)
+    vals = np.ascontiguousarray(vals).view(np.uint16)
+    o2, r2, v2 = np.empty_like(offsets), np.empty_like(rc), np.empty_like(vals)
+    _check(_lib.qlinear_pack_tilecoo(_np_ptr(offsets), _np_ptr(rc), _np_ptr(vals), N, K,
+                                     _np_ptr(o2), _np_ptr(r2), _np_ptr(v2)), "qlinear_pack_tilecoo")
+    return o2, r2, v2.view(np.float16)
+
+
+# ---------------------------------------------------------------------------
+# workspace / plan
+
+
+def qlinear_workspace_bytes(fmt: int, M: int, N: int, K: int) -> int:
+    return int(_lib.qlinear_workspace_bytes(fmt, M, N, K))
+
+
+def qlinear_plan(fmt: int, M: int, N: int, K: int) -> ql_plan:
+    p = ql_plan()
+    _check(_lib.qlinear_plan(fmt, M, N, K, ctypes.byref(p)), "qlinear_plan")
+    return p
+
+
+# ---------------------------------------------------------------------------
+# hot path (torch tensors on the current device)
+
+
+def _uniform(name, x, qweight, scales, zeros, y, M, N, K, workspace, stream, group=128):
+    st = getattr(_lib, name)(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(y), M, N, K,
+                             group, _ptr(workspace), workspace.numel() * workspace.element_size()
+                             if workspace is not None else 0, _stream(stream))
+    _check(st, name)
+    return y
+
+
+def qlinear_w4a16(x, qweight, scales, zeros, y, M, N, K, workspace, stream=None, group=128):
+    return _uniform("qlinear_w4a16", x, qweight, scales, zeros, y, M, N, K, workspace, stream, group)
+
+
+def qlinear_w2a16(x, qweight, scales, zeros, y, M, N, K, workspace, stream=None, group=128):
+    return _uniform("qlinear_w2a16", x, qweight, scales, zeros, y, M, N, K, workspace, stream, group)
+
+
+def qlinear_w8a16(x, qweight, scales, zeros, y, M, N, K, workspace, stream=None, group=128):
+    return _uniform("qlinear_w8a16", x, qweight, scales, zeros, y, M, N, K, workspace, stream, group)
+
+
+def qlinear_lut4(x, codes, lut16, absmax, y, M, N, K, workspace, stream=None, block=64):
+    st = _lib.qlinear_lut4(_ptr(x), _ptr(codes), _ptr(lut16), _ptr(absmax), _ptr(y), M, N, K, block,
+                           _ptr(workspace), workspace.numel() * workspace.element_size()
+                           if workspace is not None else 0, _stream(stream))
+    _check(st, "qlinear_lut4")
+    return y
+
+
+def qlinear_w4a16_outlier(x, qweight, scales, zeros, tile_offsets, tile_rc, tile_vals, y, M, N, K,
+                          workspace, stream=None, group=128):
+    st = _lib.qlinear_w4a16_outlier(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros),
+                                    _ptr(tile_offsets), _ptr(tile_rc), _ptr(tile_vals), _ptr(y),
+                                    M, N, K, group, _ptr(workspace),
+                                    workspace.numel() * workspace.element_size()
+                                    if workspace is not None else 0, _stream(stream))
+    _check(st, "qlinear_w4a16_outlier")
+    return y
+
+
+def qlinear_debug_unpack(fmt, packed, codes, N, K, stream=None):
+    _check(_lib.qlinear_debug_unpack(fmt, _ptr(packed), _ptr(codes), N, K, _stream(stream)),
+           "qlinear_debug_unpack")
+    return codes
+
+
+def qlinear_debug_dequant(fmt, packed, p0, p1, w, N, K, stream=None):
+    _check(_lib.qlinear_debug_dequant(fmt, _ptr(packed), _ptr(p0), _ptr(p1), _ptr(w), N, K,
+                                      _stream(stream)), "qlinear_debug_dequant")
+    return w

@@ -1,0 +1,143 @@
+// Host-side packer: canonical code / parameter / Tile-COO layouts -> kernel layout.
+// Plain C++ on host memory, no CUDA calls.  The layout itself is described in layout.h.
+#include <stdint.h>
+#include <string.h>
+
+#include <vector>
+
+#include "layout.h"
+#include "qlinear.h"
+
+using namespace qlayout;
+
+namespace {
+
+bool fmt_ok(int fmt) { return fmt == kW2 || fmt == kW4 || fmt == kW8 || fmt == kLUT4; }
+
+bool shape_ok(int N, int K) {
+  return N >= kTileN && K >= kGroup && N % kTileN == 0 && K % kGroup == 0;
+}
+
+// Code of weight (k, n) in the canonical layout.
+inline uint32_t canonical_code(int fmt, const void* canon, int N, int k, int n) {
+  if (fmt == kLUT4) {
+    const uint8_t* b = static_cast<const uint8_t*>(canon);
+    const uint8_t v = b[(size_t)(k >> 1) * N + n];
+    return (k & 1) ? (v >> 4) : (v & 0xF);
+  }
+  const int bits = fmt;
+  const int P = 32 / bits;
+  const uint32_t* w = static_cast<const uint32_t*>(canon);
+  const uint32_t v = w[(size_t)(k / P) * N + n];
+  return (v >> (bits * (k % P))) & ((1u << bits) - 1);
+}
+
+}  // namespace
+
+extern "C" size_t qlinear_packed_bytes(int fmt, int N, int K) {
+  if (!fmt_ok(fmt) || !shape_ok(N, K)) return 0;
+  return (size_t)N * K * code_bits(fmt) / 8;
+}
+
+extern "C" size_t qlinear_params_bytes(int fmt, int N, int K) {
+  if (!fmt_ok(fmt) || !shape_ok(N, K)) return 0;
+  if (fmt == kLUT4) return (size_t)(K / kLutBlock) * N * sizeof(float);
+  return (size_t)(K / kGroup) * N * sizeof(uint16_t);
+}
+
+extern "C" ql_status qlinear_pack(int fmt, const void* canonical, void* packed, int N, int K) {
+  if (!fmt_ok(fmt)) return QL_ERR_UNSUPPORTED;
+  if (!canonical || !packed) return QL_ERR_NULL;
+  if (!shape_ok(N, K)) return QL_ERR_SHAPE;
+  const int G = K / kGroup;
+  const int ntiles = N / kTileN;
+  const int nblocks = (ntiles + kBlockTiles - 1) / kBlockTiles;
+  const int WL = words_per_lane(fmt);
+  uint32_t* out = static_cast<uint32_t*>(packed);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int b = 0; b < nblocks; ++b) {
+    const int tb = tiles_in_block(b, ntiles);
+    for (int g = 0; g < G; ++g) {
+      for (int jj = 0; jj < tb; ++jj) {
+        uint32_t* chunk = out + chunk_index(b, g, jj, G, ntiles) * 32 * WL;
+        const int n_base = (b * kBlockTiles + jj) * kTileN;
+        for (int lane = 0; lane < 32; ++lane) {
+          const int gi = lane >> 2, t = lane & 3;
+          uint32_t words[16] = {0};
+          for (int s = 0; s < 8; ++s)
+            for (int dk = 0; dk < 4; ++dk)
+              for (int r8 = 0; r8 <= 8; r8 += 8) {
+                const int k = g * kGroup + k_in_group(s, t, dk);
+                const int n = n_base + gi + r8;
+                int wi, bit;
+                code_position(fmt, s, dk, r8, &wi, &bit);
+                words[wi] |= canonical_code(fmt, canonical, N, k, n) << bit;
+              }
+          memcpy(chunk + lane * WL, words, sizeof(uint32_t) * WL);
+        }
+      }
+    }
+  }
+  return QL_OK;
+}
+
+extern "C" ql_status qlinear_pack_params(int fmt, const void* canonical, void* packed, int N, int K) {
+  if (!fmt_ok(fmt)) return QL_ERR_UNSUPPORTED;
+  if (!canonical || !packed) return QL_ERR_NULL;
+  if (!shape_ok(N, K)) return QL_ERR_SHAPE;
+  const int G = K / kGroup;
+  const int ntiles = N / kTileN;
+  const int nblocks = (ntiles + kBlockTiles - 1) / kBlockTiles;
+  for (int b = 0; b < nblocks; ++b) {
+    const int tb = tiles_in_block(b, ntiles);
+    for (int g = 0; g < G; ++g)
+      for (int jj = 0; jj < tb; ++jj) {
+        const long long c = chunk_index(b, g, jj, G, ntiles);
+        const int n_base = (b * kBlockTiles + jj) * kTileN;
+        for (int gi = 0; gi < 8; ++gi)
+          for (int h = 0; h < 2; ++h) {
+            const int n = n_base + gi + 8 * h;
+            if (fmt == kLUT4) {
+              const float* a = static_cast<const float*>(canonical);
+              float* o = static_cast<float*>(packed);
+              for (int blk = 0; blk < 2; ++blk)
+                o[c * 32 + gi * 4 + blk * 2 + h] = a[(size_t)(2 * g + blk) * N + n];
+            } else {
+              const uint16_t* a = static_cast<const uint16_t*>(canonical);
+              uint16_t* o = static_cast<uint16_t*>(packed);
+              o[c * 16 + gi * 2 + h] = a[(size_t)g * N + n];
+            }
+          }
+      }
+  }
+  return QL_OK;
+}
+
+// Reorder Tile-COO tiles from the canonical K-major tile order (t = kt * NB + nt) to
+// the order the fused kernel walks them (t' = nt * (K / 128) + kt), so the outliers
+// of one run of work units are contiguous.  Entries keep their in-tile order.
+extern "C" ql_status qlinear_pack_tilecoo(const uint32_t* offsets, const uint8_t* rc,
+                                          const uint16_t* vals, int N, int K,
+                                          uint32_t* offsets_out, uint8_t* rc_out,
+                                          uint16_t* vals_out) {
+  if (!offsets || !rc || !vals || !offsets_out || !rc_out || !vals_out) return QL_ERR_NULL;
+  if (N <= 0 || K <= 0 || N % 128 || K % 128) return QL_ERR_SHAPE;
+  const int NB = N / 128, KT = K / 128;
+  const long long T = (long long)NB * KT;
+  if (offsets[0] != 0) return QL_ERR_SHAPE;
+  for (long long t = 0; t < T; ++t)
+    if (offsets[t + 1] < offsets[t]) return QL_ERR_SHAPE;
+  uint32_t pos = 0;
+  offsets_out[0] = 0;
+  for (int nt = 0; nt < NB; ++nt)
+    for (int kt = 0; kt < KT; ++kt) {
+      const long long t = (long long)kt * NB + nt;
+      const uint32_t b = offsets[t], e = offsets[t + 1];
+      const uint32_t n = e - b;
+      memcpy(rc_out + 2 * (size_t)pos, rc + 2 * (size_t)b, 2 * (size_t)n);
+      memcpy(vals_out + pos, vals + b, sizeof(uint16_t) * n);
+      pos += n;
+      offsets_out[(long long)nt * KT + kt + 1] = pos;
+    }
+  return QL_OK;
+}

@@ -1,0 +1,363 @@
+// C ABI of the quantized GEMV library: argument checks, launch planning, kernel
+// instances and the debug decode kernels.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#include <mutex>
+#include <unordered_map>
+
+#include "kernels.cuh"
+#include "qlinear.h"
+
+using namespace qlayout;
+
+namespace {
+
+// Kernel configuration: warps per CTA x tiles per warp = 8 tiles = one 128-column block.
+constexpr int kT = 2;
+constexpr int kW = 4;
+constexpr int kD = 2;
+constexpr int kMaxCtasPerSm = 8;
+
+bool fmt_ok(int fmt) { return fmt == kW2 || fmt == kW4 || fmt == kW8 || fmt == kLUT4; }
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Plan {
+  int C;            // CTAs
+  long long U;      // units
+  int nblocks, ntiles, G, MT;
+  size_t partial_bytes, counter_offset, ws_bytes;
+};
+
+using KernelPtr = void (*)(qlk::GemvParams);
+
+template <int FMT, int MT, bool OUTL>
+KernelPtr kernel_ptr() {
+  return qlk::qgemv_kernel<FMT, MT, kT, kW, kD, OUTL>;
+}
+
+KernelPtr select_kernel(int fmt, int MT, bool outl) {
+  if (outl) return MT == 1 ? kernel_ptr<kW4, 1, true>() : kernel_ptr<kW4, 2, true>();
+  switch (fmt) {
+    case kW2: return MT == 1 ? kernel_ptr<kW2, 1, false>() : kernel_ptr<kW2, 2, false>();
+    case kW4: return MT == 1 ? kernel_ptr<kW4, 1, false>() : kernel_ptr<kW4, 2, false>();
+    case kW8: return MT == 1 ? kernel_ptr<kW8, 1, false>() : kernel_ptr<kW8, 2, false>();
+    default: return MT == 1 ? kernel_ptr<kLUT4, 1, false>() : kernel_ptr<kLUT4, 2, false>();
+  }
+}
+
+// Resident CTAs per SM of a kernel on a device (queried once, then cached).
+cudaError_t ctas_per_sm(KernelPtr k, int dev, int* out) {
+  static std::mutex mu;
+  static std::unordered_map<uint64_t, int> cache;
+  const uint64_t key = ((uint64_t)(uintptr_t)k << 8) ^ (uint64_t)dev;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *out = it->second;
+      return cudaSuccess;
+    }
+  }
+  int occ = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kW * 32, 0);
+  if (e != cudaSuccess) return e;
+  if (occ < 1) occ = 1;
+  if (occ > kMaxCtasPerSm) occ = kMaxCtasPerSm;
+  std::lock_guard<std::mutex> lk(mu);
+  cache[key] = occ;
+  *out = occ;
+  return cudaSuccess;
+}
+
+cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  p->MT = M <= 8 ? 1 : 2;
+  int occ = 1;
+  e = ctas_per_sm(select_kernel(fmt, p->MT, outl), dev, &occ);
+  if (e != cudaSuccess) return e;
+  p->G = K / kGroup;
+  p->ntiles = N / kTileN;
+  p->nblocks = (p->ntiles + kBlockTiles - 1) / kBlockTiles;
+  p->U = (long long)p->nblocks * p->G;
+  long long C = (long long)sms * occ;
+  // QLINEAR_MAX_CTAS caps the persistent grid (A/B runs, tests of the split-K fix-up)
+  if (const char* cap = getenv("QLINEAR_MAX_CTAS")) {
+    const long long v = atoll(cap);
+    if (v > 0 && v < C) C = v;
+  }
+  if (C > p->U) C = p->U;
+  p->C = (int)C;
+  p->partial_bytes = (size_t)2 * p->C * kW * kT * 32 * 4 * p->MT * sizeof(float);
+  p->counter_offset = align_up(p->partial_bytes, 256);
+  p->ws_bytes = p->counter_offset + align_up((size_t)p->nblocks * kW * sizeof(uint32_t), 256);
+  return cudaSuccess;
+}
+
+bool shape_ok(int M, int N, int K) {
+  return M >= 1 && M <= 16 && N >= kTileN && K >= kGroup && N % kTileN == 0 && K % kGroup == 0;
+}
+
+struct Call {
+  int fmt;
+  bool outl;
+  const void* x;
+  const void* qw;
+  const void* p0;
+  const void* p1;
+  const uint32_t* toff;
+  const uint8_t* trc;
+  const uint16_t* tval;
+  void* y;
+  int M, N, K;
+  void* ws;
+  size_t ws_bytes;
+  cudaStream_t stream;
+};
+
+ql_status run(const Call& c) {
+  if (!c.x || !c.qw || !c.p0 || !c.p1 || !c.y) return QL_ERR_NULL;
+  if (c.outl && (!c.toff || !c.trc || !c.tval)) return QL_ERR_NULL;
+  if (!shape_ok(c.M, c.N, c.K)) return QL_ERR_SHAPE;
+  if (c.outl && (c.N % 128 || c.K / kGroup > qlk::kMaxOutlierGroups)) return QL_ERR_SHAPE;
+  if (!aligned(c.x, 16) || !aligned(c.qw, 32) || !aligned(c.y, 2)) return QL_ERR_ALIGN;
+  if (c.fmt == kLUT4) {
+    if (!aligned(c.p0, 2) || !aligned(c.p1, 16)) return QL_ERR_ALIGN;
+  } else if (!aligned(c.p0, 4) || !aligned(c.p1, 4)) {
+    return QL_ERR_ALIGN;
+  }
+  if (c.outl && (!aligned(c.toff, 4) || !aligned(c.trc, 2) || !aligned(c.tval, 2)))
+    return QL_ERR_ALIGN;
+  Plan p;
+  if (make_plan(c.fmt, c.M, c.N, c.K, c.outl, &p) != cudaSuccess) return QL_ERR_CUDA;
+  if (!c.ws || c.ws_bytes < p.ws_bytes) return QL_ERR_WORKSPACE;
+  if (!aligned(c.ws, 16)) return QL_ERR_ALIGN;
+  qlk::GemvParams P;
+  P.x = static_cast<const __half*>(c.x);
+  P.qw = static_cast<const uint8_t*>(c.qw);
+  P.sc = static_cast<const __half*>(c.p0);
+  P.zp = c.p1;
+  P.tile_off = c.toff;
+  P.tile_rc = reinterpret_cast<const uint16_t*>(c.trc);
+  P.tile_val = c.tval;
+  P.y = static_cast<__half*>(c.y);
+  P.partials = static_cast<float*>(c.ws);
+  P.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(c.ws) + p.counter_offset);
+  P.M = c.M;
+  P.N = c.N;
+  P.K = c.K;
+  P.G = p.G;
+  P.nblocks = p.nblocks;
+  P.ntiles = p.ntiles;
+  P.U = p.U;
+  P.C = p.C;
+  KernelPtr k = select_kernel(c.fmt, p.MT, c.outl);
+  k<<<p.C, kW * 32, 0, c.stream>>>(P);
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// debug decode kernels: one warp per chunk, same fragment extraction as the GEMV
+
+template <int FMT>
+__device__ __forceinline__ uint32_t field_shift(int s, int r) {
+  if constexpr (FMT == kW4) return (r & 1) ? 4u : 0u;
+  if constexpr (FMT == kW2) return 4u * (s & 1) + ((r & 1) ? 2u : 0u);
+  return 0u;
+}
+
+template <int FMT, bool DEQ>
+__global__ void __launch_bounds__(128) debug_kernel(const uint8_t* packed, const void* p0,
+                                                    const void* p1, uint8_t* codes, float* w,
+                                                    int N, int K) {
+  __shared__ uint32_t tbl[FMT == kLUT4 ? 256 * 32 : 1];
+  const int G = K / kGroup, ntiles = N / kTileN;
+  if constexpr (FMT == kLUT4 && DEQ) {
+    qlk::build_lut_table(tbl, static_cast<const __half*>(p0), threadIdx.x, 128);
+    __syncthreads();
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long id = (long long)blockIdx.x * 4 + warp;
+  if (id >= (long long)ntiles * G) return;
+  const int g = (int)(id % G), j = (int)(id / G);
+  const int b = j / kBlockTiles, jj = j % kBlockTiles;
+  const long long ch = chunk_index(b, g, jj, G, ntiles);
+  constexpr int KW = qlk::Fmt<FMT>::kWords;
+  uint32_t wv[KW];
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(packed + ch * chunk_bytes(FMT)) + lane * KW;
+#pragma unroll
+  for (int i = 0; i < KW; ++i) wv[i] = src[i];
+  const int gi = lane >> 2, t4 = lane & 3;
+  float2 s2 = make_float2(0.f, 0.f), z2 = s2;
+  float4 am = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (DEQ) {
+    if constexpr (FMT == kLUT4) {
+      am = *reinterpret_cast<const float4*>(static_cast<const float*>(p1) + ch * 32 + gi * 4);
+    } else {
+      s2 = __half22float2(*reinterpret_cast<const __half2*>(static_cast<const __half*>(p0) + ch * 16 + gi * 2));
+      z2 = __half22float2(*reinterpret_cast<const __half2*>(static_cast<const __half*>(p1) + ch * 16 + gi * 2));
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    uint32_t a[4];
+    if constexpr (FMT == kLUT4) {
+      if (DEQ) qlk::frag_lut(wv[s], tbl, lane, a);
+      else a[0] = a[1] = a[2] = a[3] = 0u;
+    } else {
+      qlk::frag_uniform<FMT>(wv, s, a);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int row = gi + 8 * (r & 1);
+        const int dk = e + 2 * (r >> 1);
+        const int k = g * kGroup + k_in_group(s, t4, dk);
+        const int n = j * kTileN + row;
+        const __half hv = __ushort_as_half((unsigned short)(a[r] >> (16 * e)));
+        if constexpr (FMT == kLUT4) {
+          const uint32_t byte = (wv[s] >> (8 * r)) & 0xFFu;
+          const uint32_t q = e ? (byte >> 4) : (byte & 0xFu);
+          if (DEQ) {
+            const float amv = (s >= 4) ? ((r & 1) ? am.w : am.z) : ((r & 1) ? am.y : am.x);
+            w[(size_t)k * N + n] = __fmul_rn(__half2float(hv), amv);
+          } else {
+            codes[(size_t)k * N + n] = (uint8_t)q;
+          }
+        } else {
+          // the fp16 value is code * 2^(shift - 24): decode it numerically
+          const uint32_t iv = (uint32_t)(__half2float(hv) * 16777216.0f);
+          const uint32_t q = iv >> field_shift<FMT>(s, r);
+          if (DEQ) {
+            const float sc = (r & 1) ? s2.y : s2.x, zc = (r & 1) ? z2.y : z2.x;
+            w[(size_t)k * N + n] = __fmul_rn(sc, (float)q - zc);
+          } else {
+            codes[(size_t)k * N + n] = (uint8_t)q;
+          }
+        }
+      }
+  }
+}
+
+template <bool DEQ>
+ql_status launch_debug(int fmt, const void* packed, const void* p0, const void* p1,
+                       uint8_t* codes, float* w, int N, int K, cudaStream_t st) {
+  const long long chunks = (long long)(N / kTileN) * (K / kGroup);
+  const unsigned grid = (unsigned)((chunks + 3) / 4);
+  switch (fmt) {
+    case kW2: debug_kernel<kW2, DEQ><<<grid, 128, 0, st>>>(static_cast<const uint8_t*>(packed), p0, p1, codes, w, N, K); break;
+    case kW4: debug_kernel<kW4, DEQ><<<grid, 128, 0, st>>>(static_cast<const uint8_t*>(packed), p0, p1, codes, w, N, K); break;
+    case kW8: debug_kernel<kW8, DEQ><<<grid, 128, 0, st>>>(static_cast<const uint8_t*>(packed), p0, p1, codes, w, N, K); break;
+    default: debug_kernel<kLUT4, DEQ><<<grid, 128, 0, st>>>(static_cast<const uint8_t*>(packed), p0, p1, codes, w, N, K); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// exported entry points
+
+extern "C" const char* ql_status_str(int status) {
+  switch (status) {
+    case QL_OK: return "ok";
+    case QL_ERR_NULL: return "null pointer argument";
+    case QL_ERR_SHAPE: return "unsupported shape (M in 1..16, N % 16 == 0, K % 128 == 0, group 128, block 64)";
+    case QL_ERR_ALIGN: return "misaligned pointer";
+    case QL_ERR_UNSUPPORTED: return "unknown format";
+    case QL_ERR_WORKSPACE: return "workspace missing or too small";
+    case QL_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+extern "C" size_t qlinear_workspace_bytes(int fmt, int M, int N, int K) {
+  if (!fmt_ok(fmt) || !shape_ok(M, N, K)) return 0;
+  Plan p;
+  if (make_plan(fmt, M, N, K, false, &p) != cudaSuccess) return 0;
+  // the outlier kernel (W4) may resolve to a different occupancy: cover both
+  if (fmt == kW4 && N % 128 == 0) {
+    Plan q;
+    if (make_plan(fmt, M, N, K, true, &q) == cudaSuccess && q.ws_bytes > p.ws_bytes) return q.ws_bytes;
+  }
+  return p.ws_bytes;
+}
+
+extern "C" ql_status qlinear_plan(int fmt, int M, int N, int K, ql_plan* plan) {
+  if (!plan) return QL_ERR_NULL;
+  if (!fmt_ok(fmt)) return QL_ERR_UNSUPPORTED;
+  if (!shape_ok(M, N, K)) return QL_ERR_SHAPE;
+  Plan p;
+  if (make_plan(fmt, M, N, K, false, &p) != cudaSuccess) return QL_ERR_CUDA;
+  plan->ctas = p.C;
+  plan->warps = kW;
+  plan->tiles_per_warp = kT;
+  plan->units = p.U;
+  plan->m_bucket = p.MT;
+  return QL_OK;
+}
+
+#define QL_UNIFORM_ENTRY(NAME, FMT)                                                              \
+  extern "C" ql_status NAME(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,  \
+                            const uint16_t* zeros, uint16_t* y, int M, int N, int K, int group,  \
+                            void* workspace, size_t workspace_bytes, ql_stream_t stream) {       \
+    if (group != kGroup) return QL_ERR_SHAPE;                                                     \
+    Call c{FMT, false, x, qweight, scales, zeros, nullptr, nullptr, nullptr, y, M, N, K,         \
+           workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)};                   \
+    return run(c);                                                                                \
+  }
+
+QL_UNIFORM_ENTRY(qlinear_w4a16, kW4)
+QL_UNIFORM_ENTRY(qlinear_w2a16, kW2)
+QL_UNIFORM_ENTRY(qlinear_w8a16, kW8)
+
+extern "C" ql_status qlinear_lut4(const uint16_t* x, const uint8_t* codes, const uint16_t* lut16,
+                                  const float* absmax, uint16_t* y, int M, int N, int K, int block,
+                                  void* workspace, size_t workspace_bytes, ql_stream_t stream) {
+  if (block != kLutBlock) return QL_ERR_SHAPE;
+  Call c{kLUT4, false, x, codes, lut16, absmax, nullptr, nullptr, nullptr, y, M, N, K,
+         workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)};
+  return run(c);
+}
+
+extern "C" ql_status qlinear_w4a16_outlier(const uint16_t* x, const uint32_t* qweight,
+                                           const uint16_t* scales, const uint16_t* zeros,
+                                           const uint32_t* tile_offsets, const uint8_t* tile_rc,
+                                           const uint16_t* tile_vals, uint16_t* y, int M, int N,
+                                           int K, int group, void* workspace,
+                                           size_t workspace_bytes, ql_stream_t stream) {
+  if (group != kGroup) return QL_ERR_SHAPE;
+  Call c{kW4, true, x, qweight, scales, zeros, tile_offsets, tile_rc, tile_vals, y, M, N, K,
+         workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)};
+  return run(c);
+}
+
+extern "C" ql_status qlinear_debug_unpack(int fmt, const void* packed, uint8_t* codes, int N,
+                                          int K, ql_stream_t stream) {
+  if (!fmt_ok(fmt)) return QL_ERR_UNSUPPORTED;
+  if (!packed || !codes) return QL_ERR_NULL;
+  if (!shape_ok(1, N, K)) return QL_ERR_SHAPE;
+  if (!aligned(packed, 16)) return QL_ERR_ALIGN;
+  return launch_debug<false>(fmt, packed, nullptr, nullptr, codes, nullptr, N, K,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" ql_status qlinear_debug_dequant(int fmt, const void* packed, const void* p0,
+                                           const void* p1, float* w, int N, int K,
+                                           ql_stream_t stream) {
+  if (!fmt_ok(fmt)) return QL_ERR_UNSUPPORTED;
+  if (!packed || !p0 || !p1 || !w) return QL_ERR_NULL;
+  if (!shape_ok(1, N, K)) return QL_ERR_SHAPE;
+  if (!aligned(packed, 16) || !aligned(w, 4)) return QL_ERR_ALIGN;
+  if (fmt == kLUT4 ? !aligned(p1, 16) : (!aligned(p0, 4) || !aligned(p1, 4))) return QL_ERR_ALIGN;
+  return launch_debug<true>(fmt, packed, p0, p1, nullptr, w, N, K,
+                            reinterpret_cast<cudaStream_t>(stream));
+}

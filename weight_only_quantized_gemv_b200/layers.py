@@ -1,0 +1,106 @@
+"""Device-resident quantized linear layers.
+
+A layer takes the canonical arrays of one weight matrix (NumPy, host), packs them
+with the library's host packer, uploads the packed arrays once, and owns a
+zero-filled workspace.  ``forward`` enqueues the entry point on a stream.  The
+class only moves and marshals data; every operation runs in ``libqlinear.so``.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import (QL_FMT_LUT4, QL_FMT_W2, QL_FMT_W4, QL_FMT_W8, qlinear_debug_dequant,
+               qlinear_debug_unpack, qlinear_lut4, qlinear_pack, qlinear_pack_params,
+               qlinear_pack_tilecoo, qlinear_w2a16, qlinear_w4a16, qlinear_w4a16_outlier,
+               qlinear_w8a16, qlinear_workspace_bytes)
+
+_ENTRY = {QL_FMT_W2: qlinear_w2a16, QL_FMT_W4: qlinear_w4a16, QL_FMT_W8: qlinear_w8a16}
+
+
+def _dev(a: np.ndarray, device) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+class QuantLinear:
+    """One quantized weight matrix [K, N] resident on a CUDA device."""
+
+    def __init__(self, fmt: int, K: int, N: int, canonical_codes: np.ndarray,
+                 p0: np.ndarray, p1: Optional[np.ndarray] = None,
+                 tilecoo: Optional[tuple] = None, device="cuda", max_m: int = 16):
+        self.fmt, self.K, self.N = fmt, K, N
+        self.device = torch.device(device)
+        packed = qlinear_pack(fmt, canonical_codes, N, K)
+        self.qweight = _dev(packed, self.device)
+        if fmt == QL_FMT_LUT4:
+            self.p0 = _dev(np.asarray(p0, dtype=np.float16).view(np.uint16), self.device)  # lut16
+            self.p1 = _dev(qlinear_pack_params(fmt, np.asarray(p1, dtype=np.float32), N, K),
+                           self.device)  # absmax
+        else:
+            self.p0 = _dev(qlinear_pack_params(fmt, np.asarray(p0, dtype=np.float16), N, K)
+                           .view(np.uint16), self.device)  # scales
+            self.p1 = _dev(qlinear_pack_params(fmt, np.asarray(p1, dtype=np.float16), N, K)
+                           .view(np.uint16), self.device)  # zeros
+        self.tile = None
+        if tilecoo is not None:
+            off, rc, vals = qlinear_pack_tilecoo(*tilecoo, N, K)
+            self.tile = (_dev(off, self.device), _dev(rc, self.device),
+                         _dev(vals.view(np.uint16), self.device))
+        ws = max(qlinear_workspace_bytes(fmt, m, N, K) for m in (1, max_m))
+        self.workspace = torch.zeros(max(ws, 256) // 4 + 64, dtype=torch.int32, device=self.device)
+
+    @property
+    def weight_bytes(self) -> int:
+        b = self.qweight.numel() + self.p0.numel() * self.p0.element_size() + \
+            self.p1.numel() * self.p1.element_size()
+        if self.tile is not None:
+            b += sum(t.numel() * t.element_size() for t in self.tile)
+        return b
+
+    def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """y[M, N] (fp16) = x[M, K] (fp16) . W."""
+        M = x.shape[0]
+        if y is None:
+            y = torch.empty((M, self.N), dtype=torch.float16, device=self.device)
+        xv = x.view(torch.int16)
+        yv = y.view(torch.int16)
+        if self.tile is not None:
+            qlinear_w4a16_outlier(xv, self.qweight, self.p0, self.p1, *self.tile, yv, M, self.N,
+                                  self.K, self.workspace, stream)
+        elif self.fmt == QL_FMT_LUT4:
+            qlinear_lut4(xv, self.qweight, self.p0, self.p1, yv, M, self.N, self.K,
+                         self.workspace, stream)
+        else:
+            _ENTRY[self.fmt](xv, self.qweight, self.p0, self.p1, yv, M, self.N, self.K,
+                             self.workspace, stream)
+        return y
+
+    def debug_unpack(self, stream=None) -> torch.Tensor:
+        codes = torch.empty((self.K, self.N), dtype=torch.uint8, device=self.device)
+        qlinear_debug_unpack(self.fmt, self.qweight, codes, self.N, self.K, stream)
+        return codes
+
+    def debug_dequant(self, stream=None) -> torch.Tensor:
+        w = torch.empty((self.K, self.N), dtype=torch.float32, device=self.device)
+        qlinear_debug_dequant(self.fmt, self.qweight, self.p0, self.p1, w, self.N, self.K, stream)
+        return w
+
+
+def from_uniform(layer, device="cuda", max_m: int = 16) -> QuantLinear:
+    """From a ``synth.gen.UniformLayer``-like object (bits, K, N, qweight, scales, zeros)."""
+    return QuantLinear(layer.bits, layer.K, layer.N, layer.qweight, layer.scales, layer.zeros,
+                       device=device, max_m=max_m)
+
+
+def from_lut4(layer, device="cuda", max_m: int = 16) -> QuantLinear:
+    return QuantLinear(QL_FMT_LUT4, layer.K, layer.N, layer.qbytes, layer.lut, layer.absmax,
+                       device=device, max_m=max_m)
+
+
+def from_outlier(layer, device="cuda", max_m: int = 16) -> QuantLinear:
+    d = layer.dense
+    return QuantLinear(QL_FMT_W4, d.K, d.N, d.qweight, d.scales, d.zeros,
+                       tilecoo=(layer.tile_offsets, layer.tile_rc, layer.tile_vals),
+                       device=device, max_m=max_m)
