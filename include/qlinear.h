@@ -114,8 +114,16 @@ ql_status qlinear_pack_tilecoo(const uint32_t* offsets, const uint8_t* rc, const
  * the counters at zero again, so no per-call clearing is needed.
  * ------------------------------------------------------------------------- */
 
-/* Workspace bytes for a call with these arguments on the current device; 0 if none. */
+/* Workspace bytes for a call with these arguments on the current device; 0 for invalid
+ * arguments or when no CUDA device is available. */
 size_t qlinear_workspace_bytes(int fmt, int M, int N, int K);
+
+/* The first 32-bit word of a workspace collects sticky error flags of the calls that used
+ * it: bit 0 = a consumer gave up waiting for a shared-memory stage, bit 1 = the producer
+ * gave up waiting for a stage to be released (each wait is bounded so that a lost copy
+ * cannot hang the GPU; results of such a call are undefined).  This call waits for
+ * `stream`, copies the word to *flags and clears it.  Synchronous. */
+ql_status qlinear_read_error(void* workspace, uint32_t* flags, ql_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Hot path (device pointers, asynchronous on `stream`).
@@ -149,7 +157,7 @@ ql_status qlinear_lut4(const uint16_t* x, const uint8_t* codes, const uint16_t* 
  * kernel.  The Tile-COO arrays are those written by qlinear_pack_tilecoo (tiles in
  * block-major order): tile_offsets uint32[T+1] (4-byte aligned), tile_rc uint8[nnz][2]
  * (2-byte aligned), tile_vals fp16[nnz] (2-byte aligned), T = (K/128) * (N/128).
- * Needs N % 128 == 0 and K <= 65536.  The dense code of every outlier position should
+ * Needs N % 128 == 0.  The dense code of every outlier position should
  * hold its group's zero code (then the dense part contributes nothing there). */
 ql_status qlinear_w4a16_outlier(const uint16_t* x, const uint32_t* qweight,
                                 const uint16_t* scales, const uint16_t* zeros,

@@ -57,6 +57,7 @@ _SIGS = {
     "qlinear_debug_unpack": (_I, [_I, _P, _P, _I, _I, _P]),
     "qlinear_debug_dequant": (_I, [_I, _P, _P, _P, _P, _I, _I, _P]),
     "qlinear_plan": (_I, [_I, _I, _I, _I, ctypes.POINTER(ql_plan)]),
+    "qlinear_read_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint32), _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -150,6 +151,14 @@ def qlinear_plan(fmt: int, M: int, N: int, K: int) -> ql_plan:
     p = ql_plan()
     _check(_lib.qlinear_plan(fmt, M, N, K, ctypes.byref(p)), "qlinear_plan")
     return p
+
+
+def qlinear_read_error(workspace, stream=None) -> int:
+    """Sticky error flags of the calls that used `workspace` (then cleared); 0 = none."""
+    flags = ctypes.c_uint32(0)
+    _check(_lib.qlinear_read_error(_ptr(workspace), ctypes.byref(flags), _stream(stream)),
+           "qlinear_read_error")
+    return int(flags.value)
 
 
 # ---------------------------------------------------------------------------

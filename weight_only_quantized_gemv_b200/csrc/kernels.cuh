@@ -9,14 +9,19 @@
 // Design (B200):
 //  * Work units are (128-column block, 128-element group) pairs, split evenly over a
 //    persistent grid of C CTAs (stream-K): CTA c owns the contiguous unit range
-//    [c U / C, (c+1) U / C).  Every CTA streams one contiguous byte range of the
-//    packed weights and the load balance is within one unit.  A range cuts at most
-//    two blocks; their partial sums meet in an fp32 workspace and the last CTA to
-//    arrive at a block (atomic counter, no waiting) adds them up in a fixed order.
-//  * Each warp owns T 16-column tiles of the block.  A lane reads its 8 K-steps of a
-//    tile-group with one 256-bit (W4, LUT4; two for W8) or 128-bit (W2) evict-first
-//    load; weights are used once, so they skip L1 and leave L2 first.  Loads run D
-//    groups ahead of the math.
+//    [c U / C, (c+1) U / C), i.e. one contiguous byte range of the packed weights.
+//    A range cuts at most two blocks; their partial sums meet in an fp32 workspace
+//    and the last CTA to arrive at a block (atomic counter, no waiting) adds them
+//    up in a fixed order.
+//  * One producer warp streams the range through a ring of S shared-memory stages
+//    with non-multicast bulk copies (cp.async.bulk, TMA 1-D): per unit the codes of
+//    the block's tiles, their scales/zeros (or absmax) and the M rows of x for the
+//    group, all completing on the stage's mbarrier.  Weights and parameters carry
+//    an L2 evict-first hint: they are read once.  Bytes in flight are bounded by
+//    shared memory, not registers.
+//  * Four consumer warps own two 16-column tiles each.  A consumer copies its part
+//    of the stage into registers (conflict-free 128-bit reads), releases the stage
+//    and does the math:
 //  * Codes become tensor-core operands with one AND each: a code in the low mantissa
 //    bits of an fp16 with zero exponent is the exact subnormal q * 2^-24 (times a
 //    power of two fixed by its bit field, undone in the epilogue).  The inner dot
@@ -29,10 +34,12 @@
 //    The epilogue is two FMAs per output per group: acc += s * (d - z * xsum).
 //  * LUT4 codes index a 256-entry table of fp16 pairs (one byte = the two codes of a
 //    fragment register) replicated 32 times in shared memory, one copy per bank.
-//  * The outlier variant adds the Tile-COO entries of each visited 128 x 128 tile into
-//    a shared fp32 y tile while the dense part streams, reusing x lines the dense
-//    path has just pulled into L1; the y tile joins the dense sums at the end of the
-//    unit range, before the split-K fix-up.
+//  * The outlier variant adds the Tile-COO entries of each unit into a shared fp32
+//    y tile, reading x from the same stage the dense path uses; the y tile joins
+//    the dense sums at the end of the unit range, before the split-K fix-up.
+//  * Every mbarrier wait is bounded.  A wait that runs out sets a bit in the
+//    workspace error word and carries on, so a lost copy can corrupt results but
+//    never hang the GPU.
 #pragma once
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -43,7 +50,10 @@ namespace qlk {
 
 using namespace qlayout;
 
-constexpr int kMaxOutlierGroups = 512;  // K <= 65536 for the outlier variant
+constexpr int kMaxUnitsPerCta = 1024;   // outlier variant: per-CTA offsets kept in smem
+constexpr uint32_t kErrFullTimeout = 1u;
+constexpr uint32_t kErrEmptyTimeout = 2u;
+constexpr uint32_t kSpinLimit = 1u << 22;  // try_wait rounds before a wait is abandoned
 
 struct GemvParams {
   const __half* x;            // [M][K]
@@ -54,11 +64,13 @@ struct GemvParams {
   const uint16_t* tile_rc;    // row | col << 8
   const uint16_t* tile_val;   // fp16 bits
   __half* y;                  // [M][N]
-  float* partials;            // split-K slots [2C][W][T][32][4 MT]
-  uint32_t* counters;         // [nblocks][W]
+  float* partials;            // split-K slots [2C][NC][T][32][4 MT]
+  uint32_t* counters;         // [nblocks][NC]
+  uint32_t* err;              // sticky error flags
   int M, N, K, G, nblocks, ntiles;
   long long U;                // nblocks * G
   int C;                      // CTAs
+  uint32_t mul_shr8;          // 2^24: v >> 8 as mul.hi on the FMA pipe (set by the host)
 };
 
 template <int FMT> struct Fmt;
@@ -66,41 +78,115 @@ template <> struct Fmt<kW4> {
   static constexpr int kWords = 8;
   static constexpr uint32_t kOnesHi = 0x00100010u;  // rows gi+8 carry a factor 16
   static constexpr float kHiScale = 1.0f / 16.0f;
+  static constexpr int kStages = 8;
 };
 template <> struct Fmt<kW2> {
   static constexpr int kWords = 4;
   static constexpr uint32_t kOnesHi = 0x00040004u;  // rows gi+8 carry a factor 4
   static constexpr float kHiScale = 1.0f / 4.0f;
+  static constexpr int kStages = 12;
 };
 template <> struct Fmt<kW8> {
   static constexpr int kWords = 16;
   static constexpr uint32_t kOnesHi = 0x00010001u;
   static constexpr float kHiScale = 1.0f;
+  static constexpr int kStages = 8;
 };
 template <> struct Fmt<kLUT4> {
   static constexpr int kWords = 8;
   static constexpr uint32_t kOnesHi = 0;
   static constexpr float kHiScale = 1.0f;
+  static constexpr int kStages = 8;
 };
 
 constexpr uint32_t kOnesLo = 0x00010001u;  // fp16 pair (2^-24, 2^-24)
 constexpr float kTwo24 = 16777216.0f;
 
-// ---------------------------------------------------------------------------
-// memory access helpers
+__host__ __device__ constexpr int align_to(int v, int a) { return (v + a - 1) / a * a; }
 
-__device__ __forceinline__ void ldg_stream(const uint8_t* p, uint32_t (&r)[8]) {
-  asm volatile(
-      "ld.global.nc.L1::no_allocate.L2::evict_first.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7])
-      : "l"(p));
+// Shared-memory layout of one kernel instance.
+template <int FMT, int MT, bool OUTL>
+struct Cfg {
+  static constexpr int NC = 4;                       // consumer warps
+  static constexpr int T = 2;                        // tiles per warp in the block epilogue
+  static constexpr int kThreads = (NC + 1) * 32;     // + one producer warp
+  static constexpr int KW = Fmt<FMT>::kWords;
+  static constexpr int NACC = 4 * MT;
+  static constexpr int S = Fmt<FMT>::kStages;        // a multiple of NC: warp w uses stages w mod NC
+  static_assert(S % NC == 0, "stages must split evenly over the consumer warps");
+  static constexpr int kChunkBytes = 128 * KW;
+  static constexpr int kCodeBytes = kBlockTiles * kChunkBytes;
+  static constexpr int kParamChunk = (FMT == kLUT4) ? 128 : 32;   // per tile, per array
+  static constexpr int kParamBytes = (FMT == kLUT4) ? 8 * 128 : 2 * 8 * 32;
+  static constexpr int kXStride = 272;                             // 256 + 16 pad (banks)
+  static constexpr int kXRows = 8 * MT;
+  static constexpr int kXOff = kCodeBytes + kParamBytes;
+  static constexpr int kStageBytes = align_to(kXOff + kXRows * kXStride, 128);
+  static constexpr int kRingBytes = S * kStageBytes;
+  static constexpr int kBarOff = kRingBytes;                       // full[S], empty[S]
+  static constexpr int kLutOff = align_to(kBarOff + 16 * S, 128);
+  static constexpr int kLutBytes = (FMT == kLUT4) ? 256 * 32 * 4 : 0;
+  static constexpr int kRedOff = kLutOff + kLutBytes;              // per-warp block sums
+  static constexpr int kRedBytes = NC * kBlockTiles * 32 * NACC * 4;
+  static constexpr int kYsmOff = kRedOff + kRedBytes;
+  static constexpr int kYsmBytes = OUTL ? 16 * 128 * 4 : 0;
+  static constexpr int kToffOff = kYsmOff + kYsmBytes;
+  static constexpr int kToffBytes = OUTL ? (kMaxUnitsPerCta + 1) * 4 : 0;
+  static constexpr int kSmemBytes = kToffOff + kToffBytes;
+};
+
+// ---------------------------------------------------------------------------
+// PTX helpers: mbarriers, bulk copies, shared loads
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-__device__ __forceinline__ void ldg_stream(const uint8_t* p, uint32_t (&r)[4], uint64_t pol) {
-  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "l"(p), "l"(pol));
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Bounded wait for the phase with parity `parity` to complete; false if abandoned.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kSpinLimit; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(pol)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
 __device__ __forceinline__ uint64_t evict_first_policy() {
@@ -109,27 +195,26 @@ __device__ __forceinline__ uint64_t evict_first_policy() {
   return pol;
 }
 
-template <int FMT>
-__device__ __forceinline__ void load_chunk(const uint8_t* p, uint32_t (&w)[Fmt<FMT>::kWords],
-                                           uint64_t pol) {
-  if constexpr (FMT == kW2) {
-    ldg_stream(p, w, pol);
-  } else if constexpr (FMT == kW8) {
-    uint32_t a[8], b[8];
-    ldg_stream(p, a);
-    ldg_stream(p + 32, b);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      w[i] = a[i];
-      w[8 + i] = b[i];
-    }
-  } else {
-    ldg_stream(p, w);
-  }
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint16_t lds16(uint32_t a) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
 }
 
-__device__ __forceinline__ uint4 ldg_x(const __half* p) {
-  return __ldg(reinterpret_cast<const uint4*>(p));
+__device__ __forceinline__ void consumer_sync(int nthreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -142,19 +227,29 @@ __device__ __forceinline__ void hmma(float* c, const uint32_t (&a)[4], uint32_t 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// c[0..3] = A * B (the accumulator input is zero)
+__device__ __forceinline__ void hmma0(float* c, const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%10,%10,%10,%10};"
+      : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+}
+
 // A fragment (a0a1, a2a3, a4a5, a6a7) of step s from a lane's words.  For the uniform
 // formats each half holds code << shift, the shift fixed per register (layout.h):
 // W4 rows gi+8 carry x16, W2 rows gi+8 carry x4 and odd steps x16.
+__device__ __forceinline__ uint32_t shr8(uint32_t v, uint32_t) { return v >> 8; }
+
 template <int FMT>
-__device__ __forceinline__ void frag_uniform(const uint32_t* w, int s, uint32_t (&a)[4]) {
+__device__ __forceinline__ void frag_uniform(const uint32_t* w, int s, uint32_t k24, uint32_t (&a)[4]) {
   if constexpr (FMT == kW4) {
-    const uint32_t v = w[s], h = v >> 8;
+    const uint32_t v = w[s], h = shr8(v, k24);
     a[0] = v & 0x000F000Fu;  // row gi,   dk 0 | dk 1
     a[1] = v & 0x00F000F0u;  // row gi+8, dk 0 | dk 1
     a[2] = h & 0x000F000Fu;  // row gi,   dk 2 | dk 3
     a[3] = h & 0x00F000F0u;  // row gi+8, dk 2 | dk 3
   } else if constexpr (FMT == kW2) {
-    const uint32_t v = w[s >> 1], h = v >> 8;
+    const uint32_t v = w[s >> 1], h = shr8(v, k24);
     const uint32_t m0 = (s & 1) ? 0x00300030u : 0x00030003u;
     const uint32_t m1 = (s & 1) ? 0x00C000C0u : 0x000C000Cu;
     a[0] = v & m0;
@@ -165,17 +260,17 @@ __device__ __forceinline__ void frag_uniform(const uint32_t* w, int s, uint32_t 
     const uint32_t v0 = w[2 * s], v1 = w[2 * s + 1];
     a[0] = v0 & 0x00FF00FFu;
     a[1] = v1 & 0x00FF00FFu;
-    a[2] = (v0 >> 8) & 0x00FF00FFu;
-    a[3] = (v1 >> 8) & 0x00FF00FFu;
+    a[2] = shr8(v0, k24) & 0x00FF00FFu;
+    a[3] = shr8(v1, k24) & 0x00FF00FFu;
   }
 }
 
 // LUT4: byte j of word s holds the two codes of fragment register j; the replicated
 // table gives the fp16 pair (lut[lo], lut[hi]) from the lane's own bank.
-__device__ __forceinline__ void frag_lut(uint32_t v, const uint32_t* tbl, int lane,
-                                         uint32_t (&a)[4]) {
+__device__ __forceinline__ void frag_lut(uint32_t v, uint32_t tbl, int lane, uint32_t (&a)[4]) {
 #pragma unroll
-  for (int j = 0; j < 4; ++j) a[j] = tbl[(((v >> (8 * j)) & 0xFFu) << 5) | (uint32_t)lane];
+  for (int j = 0; j < 4; ++j)
+    a[j] = lds32(tbl + (((((v >> (8 * j)) & 0xFFu) << 5) | (uint32_t)lane) << 2));
 }
 
 __device__ __forceinline__ void build_lut_table(uint32_t* tbl, const __half* lut16, int tid,
@@ -201,135 +296,96 @@ __host__ __device__ __forceinline__ int cta_of_unit(long long u, long long U, lo
 
 // ---------------------------------------------------------------------------
 
-template <int FMT, int MT, int T, int W, int D, bool OUTL>
+template <int FMT, int MT, bool OUTL>
 struct Gemv {
-  static constexpr int KW = Fmt<FMT>::kWords;
-  static constexpr int NACC = 4 * MT;  // accumulators per tile per lane
+  using C_ = Cfg<FMT, MT, OUTL>;
+  static constexpr int NC = C_::NC, T = C_::T, KW = C_::KW, NACC = C_::NACC, S = C_::S;
   static constexpr bool kLut = (FMT == kLUT4);
-  static constexpr int kThreads = W * 32;
+  static constexpr int kBT = kBlockTiles;
 
-  struct Buf {
-    uint32_t w[T][KW];
-    uint32_t p0[T];   // scale pair (uniform)
-    uint32_t p1[T];   // zero pair (uniform)
-    float4 am[T];     // absmax (LUT4)
-    uint4 xr[4];      // x fragment, rows gi (prefetched when MT == 1)
-    uint32_t orc;     // this thread's outlier of the tile: row | col << 8
-    uint32_t oval;    // its fp16 value
-    uint32_t oend;    // end offset of the tile's entries
-  };
-
-  struct Smem {
-    uint32_t lut[kLut ? 256 * 32 : 1];
-    float ysm[OUTL ? 16 : 1][OUTL ? 128 : 1];
-    uint32_t toff[OUTL ? kMaxOutlierGroups + 1 : 1];
-  };
-
-  __device__ static void load(const GemvParams& P, const Smem& sm, int b, int g, int ga, int tb,
-                              int warp, int lane, uint64_t pol, Buf& buf) {
+  // x fragments of one unit (rows gi and, for MT == 2, gi + 8), from the stage.
+  __device__ static void read_x(const GemvParams& P, uint32_t st, int lane, uint4 (&xr)[4],
+                                uint4 (&xr2)[4]) {
     const int gi = lane >> 2, t4 = lane & 3;
+    const uint32_t xb = st + C_::kXOff + gi * C_::kXStride + 16 * t4;
 #pragma unroll
-    for (int i = 0; i < T; ++i) {
-      const int jj = warp * T + i;
-      if (jj < tb) {
-        const long long ch = chunk_index(b, g, jj, P.G, P.ntiles);
-        load_chunk<FMT>(P.qw + ch * chunk_bytes(FMT) + lane * KW * 4, buf.w[i], pol);
-        if constexpr (kLut) {
-          buf.am[i] = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(P.zp) +
-                                                            ch * 32 + gi * 4));
-        } else {
-          buf.p0[i] = __ldg(reinterpret_cast<const uint32_t*>(P.sc + ch * 16 + gi * 2));
-          buf.p1[i] = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const __half*>(P.zp) +
-                                                              ch * 16 + gi * 2));
-        }
-      }
+    for (int p = 0; p < 4; ++p) {  // rows >= M hold zeros (filled once at kernel start)
+      xr[p] = lds128(xb + 64 * p);
+      if constexpr (MT == 2) xr2[p] = lds128(xb + 8 * C_::kXStride + 64 * p);
     }
-    if constexpr (MT == 1) {
-      if (gi < P.M && warp * T < tb) {
-        const __half* xp = P.x + (size_t)gi * P.K + (size_t)g * kGroup + 8 * t4;
+  }
+
+  // The stage bytes of four tiles (j0 .. j0 + 3) of one unit, in registers.
+  static constexpr int kQ = 4;
+  struct Quad {
+    uint32_t w[kQ][KW];
+    uint32_t p0[kQ], p1[kQ];  // scale / zero pairs (uniform)
+    float4 am[kQ];            // absmax (LUT4)
+  };
+
+  __device__ static void load_quad(uint32_t st, int j0, int lane, Quad& r) {
+    const int gi = lane >> 2;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) buf.xr[p] = ldg_x(xp + 32 * p);
+    for (int i = 0; i < kQ; ++i) {
+      const uint32_t cb = st + (j0 + i) * C_::kChunkBytes + lane * 16;
+#pragma unroll
+      for (int q = 0; q < KW / 4; ++q) {
+        const uint4 v = lds128(cb + q * 512);
+        r.w[i][4 * q + 0] = v.x;
+        r.w[i][4 * q + 1] = v.y;
+        r.w[i][4 * q + 2] = v.z;
+        r.w[i][4 * q + 3] = v.w;
+      }
+      if constexpr (kLut) {
+        const uint4 a = lds128(st + C_::kCodeBytes + (j0 + i) * 128 + gi * 16);
+        r.am[i] = make_float4(__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z),
+                              __uint_as_float(a.w));
       } else {
-#pragma unroll
-        for (int p = 0; p < 4; ++p) buf.xr[p] = make_uint4(0, 0, 0, 0);
-      }
-    }
-    if constexpr (OUTL) {
-      const uint32_t e = sm.toff[g - ga] + threadIdx.x;
-      buf.oend = sm.toff[g - ga + 1];
-      if (e < buf.oend) {
-        buf.orc = __ldg(P.tile_rc + e);
-        buf.oval = __ldg(P.tile_val + e);
+        r.p0[i] = lds32(st + C_::kCodeBytes + (j0 + i) * 32 + gi * 4);
+        r.p1[i] = lds32(st + C_::kCodeBytes + 256 + (j0 + i) * 32 + gi * 4);
       }
     }
   }
 
-  // Dense work of one group of the warp's tiles: MMAs plus the group epilogue.
-  __device__ static void compute(const GemvParams& P, const Smem& sm, int g, int tb, int warp,
-                                 int lane, const Buf& buf, float (&acc)[T][NACC]) {
-    const int gi = lane >> 2, t4 = lane & 3;
-    uint4 xr[4], xr2[4];
-    if constexpr (MT == 1) {
-#pragma unroll
-      for (int p = 0; p < 4; ++p) xr[p] = buf.xr[p];
-    } else {
-      const __half* xp = P.x + (size_t)gi * P.K + (size_t)g * kGroup + 8 * t4;
-      const __half* xp2 = xp + (size_t)8 * P.K;
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        xr[p] = gi < P.M ? ldg_x(xp + 32 * p) : make_uint4(0, 0, 0, 0);
-        xr2[p] = gi + 8 < P.M ? ldg_x(xp2 + 32 * p) : make_uint4(0, 0, 0, 0);
-      }
-    }
+  // MMAs and group epilogue of four tiles: four independent accumulator chains per step.
+  __device__ static void compute_quad(const Quad& r, int j0, int lane, uint32_t lut, uint32_t k24,
+                                      const uint4 (&xr)[4], const uint4 (&xr2)[4],
+                                      const float (&cx)[NACC], float (&acc)[kBT][NACC]) {
+    const auto& w = r.w;
     if constexpr (kLut) {
 #pragma unroll
       for (int blk = 0; blk < 2; ++blk) {
-        float c[T][NACC];
-#pragma unroll
-        for (int i = 0; i < T; ++i)
-#pragma unroll
-          for (int e = 0; e < NACC; ++e) c[i][e] = 0.f;
+        float c[kQ][NACC];
 #pragma unroll
         for (int s = 4 * blk; s < 4 * blk + 4; ++s) {
           const int p = s >> 1, h = s & 1;
           const uint32_t b0 = h ? xr[p].z : xr[p].x, b1 = h ? xr[p].w : xr[p].y;
-          uint32_t b2 = 0, b3 = 0;
-          if constexpr (MT == 2) {
-            b2 = h ? xr2[p].z : xr2[p].x;
-            b3 = h ? xr2[p].w : xr2[p].y;
-          }
 #pragma unroll
-          for (int i = 0; i < T; ++i) {
+          for (int i = 0; i < kQ; ++i) {
             uint32_t a[4];
-            frag_lut(buf.w[i][s], sm.lut, lane, a);
-            hmma(&c[i][0], a, b0, b1);
-            if constexpr (MT == 2) hmma(&c[i][4], a, b2, b3);
+            frag_lut(w[i][s], lut, lane, a);
+            const uint32_t b2 = h ? xr2[p].z : xr2[p].x, b3 = h ? xr2[p].w : xr2[p].y;
+            if (s == 4 * blk) {
+              hmma0(&c[i][0], a, b0, b1);
+              if constexpr (MT == 2) hmma0(&c[i][4], a, b2, b3);
+            } else {
+              hmma(&c[i][0], a, b0, b1);
+              if constexpr (MT == 2) hmma(&c[i][4], a, b2, b3);
+            }
           }
         }
 #pragma unroll
-        for (int i = 0; i < T; ++i) {
-          if (warp * T + i < tb) {
-            const float a0 = blk ? buf.am[i].z : buf.am[i].x;
-            const float a8 = blk ? buf.am[i].w : buf.am[i].y;
+        for (int i = 0; i < kQ; ++i) {
+          const float a0 = blk ? r.am[i].z : r.am[i].x;
+          const float a8 = blk ? r.am[i].w : r.am[i].y;
 #pragma unroll
-            for (int e = 0; e < NACC; ++e) acc[i][e] = fmaf((e & 2) ? a8 : a0, c[i][e], acc[i][e]);
-          }
+          for (int e = 0; e < NACC; ++e)
+            acc[j0 + i][e] = fmaf((e & 2) ? a8 : a0, c[i][e], acc[j0 + i][e]);
         }
       }
     } else {
-      const uint32_t kOnes[4] = {kOnesLo, Fmt<FMT>::kOnesHi, kOnesLo, Fmt<FMT>::kOnesHi};
-      float cx[NACC];
-      float c[T][NACC];
-      float co[(FMT == kW2) ? T : 1][NACC];
-#pragma unroll
-      for (int e = 0; e < NACC; ++e) cx[e] = 0.f;
-#pragma unroll
-      for (int i = 0; i < T; ++i)
-#pragma unroll
-        for (int e = 0; e < NACC; ++e) {
-          c[i][e] = 0.f;
-          if constexpr (FMT == kW2) co[i][e] = 0.f;
-        }
+      float c[kQ][NACC];
+      float co[(FMT == kW2) ? kQ : 1][NACC];
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
         const int p = s >> 1, h = s & 1;
@@ -339,15 +395,25 @@ struct Gemv {
           b2 = h ? xr2[p].z : xr2[p].x;
           b3 = h ? xr2[p].w : xr2[p].y;
         }
-        hmma(&cx[0], kOnes, b0, b1);
-        if constexpr (MT == 2) hmma(&cx[4], kOnes, b2, b3);
 #pragma unroll
-        for (int i = 0; i < T; ++i) {
+        for (int i = 0; i < kQ; ++i) {
           uint32_t a[4];
-          frag_uniform<FMT>(buf.w[i], s, a);
-          if (FMT == kW2 && h == 1) {
-            hmma(&co[i][0], a, b0, b1);
-            if constexpr (MT == 2) hmma(&co[i][4], a, b2, b3);
+          frag_uniform<FMT>(w[i], s, k24, a);
+          if constexpr (FMT == kW2) {
+            if (h == 1) {  // odd steps accumulate separately (their codes carry x16)
+              if (s == 1) {
+                hmma0(&co[i][0], a, b0, b1);
+                if constexpr (MT == 2) hmma0(&co[i][4], a, b2, b3);
+              } else {
+                hmma(&co[i][0], a, b0, b1);
+                if constexpr (MT == 2) hmma(&co[i][4], a, b2, b3);
+              }
+              continue;
+            }
+          }
+          if (s == 0) {
+            hmma0(&c[i][0], a, b0, b1);
+            if constexpr (MT == 2) hmma0(&c[i][4], a, b2, b3);
           } else {
             hmma(&c[i][0], a, b0, b1);
             if constexpr (MT == 2) hmma(&c[i][4], a, b2, b3);
@@ -355,33 +421,18 @@ struct Gemv {
         }
       }
 #pragma unroll
-      for (int i = 0; i < T; ++i) {
-        if (warp * T + i < tb) {
-          const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&buf.p0[i]));
-          const float2 z2 = __half22float2(*reinterpret_cast<const __half2*>(&buf.p1[i]));
+      for (int i = 0; i < kQ; ++i) {
+        const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&r.p0[i]));
+        const float2 z2 = __half22float2(*reinterpret_cast<const __half2*>(&r.p1[i]));
 #pragma unroll
-          for (int e = 0; e < NACC; ++e) {
-            float d = c[i][e];
-            if constexpr (FMT == kW2) d = fmaf(co[i][e], 0.0625f, d);  // odd steps carry x16
-            const float sc = (e & 2) ? s2.y : s2.x;
-            const float zc = (e & 2) ? z2.y : z2.x;
-            acc[i][e] = fmaf(sc, fmaf(-zc, cx[e], d), acc[i][e]);
-          }
+        for (int e = 0; e < NACC; ++e) {
+          float d = c[i][e];
+          if constexpr (FMT == kW2) d = fmaf(co[i][e], 0.0625f, d);  // odd steps carry x16
+          const float sc = (e & 2) ? s2.y : s2.x;
+          const float zc = (e & 2) ? z2.y : z2.x;
+          acc[j0 + i][e] = fmaf(sc, fmaf(-zc, cx[e], d), acc[j0 + i][e]);
         }
       }
-    }
-  }
-
-  // Outliers of tile (b, g): each thread takes entries threadIdx.x, +kThreads, ...
-  __device__ static void outliers(const GemvParams& P, Smem& sm, int g, int ga, const Buf& buf) {
-    const uint32_t e0 = sm.toff[g - ga] + threadIdx.x;
-    for (uint32_t e = e0; e < buf.oend; e += kThreads) {
-      const uint32_t rc = (e == e0) ? buf.orc : (uint32_t)__ldg(P.tile_rc + e);
-      const uint32_t vb = (e == e0) ? buf.oval : (uint32_t)__ldg(P.tile_val + e);
-      const int r = rc & 0xFF, col = rc >> 8;
-      const float v = __half2float(__ushort_as_half((unsigned short)vb));
-      const __half* xc = P.x + (size_t)g * kGroup + r;
-      for (int m = 0; m < P.M; ++m) atomicAdd(&sm.ysm[m][col], v * __half2float(xc[(size_t)m * P.K]));
     }
   }
 
@@ -402,47 +453,47 @@ struct Gemv {
     }
   }
 
-  __device__ static void segment(const GemvParams& P, Smem& sm, int b, int ga, int gb,
-                                 int first_block, int warp, int lane, uint64_t pol) {
+  // End of a run of units of block b: combine the warps' sums (each warp then owns
+  // tiles 2w, 2w+1), rescale, add outliers, write y or join the split-K fix-up.
+  __device__ static void finish_block(const GemvParams& P, uint8_t* smem, int b, bool whole,
+                                      int first_block, int warp, int lane,
+                                      float (&acc)[kBT][NACC]) {
     const int tb = tiles_in_block(b, P.ntiles);
-    float acc[T][NACC];
+    float* red = reinterpret_cast<float*>(smem + C_::kRedOff);
+    float* ysm = reinterpret_cast<float*>(smem + C_::kYsmOff);
+    consumer_sync(NC * 32);  // all units of the run are done (and their outliers in ysm)
 #pragma unroll
-    for (int i = 0; i < T; ++i)
+    for (int j = 0; j < kBT; ++j) {
 #pragma unroll
-      for (int e = 0; e < NACC; ++e) acc[i][e] = 0.f;
-
-    if constexpr (OUTL) {
-      for (int i = threadIdx.x; i <= gb - ga; i += kThreads)
-        sm.toff[i] = __ldg(P.tile_off + (long long)b * P.G + ga + i);
-      __syncthreads();
+      for (int e = 0; e < NACC; e += 4)
+        *reinterpret_cast<float4*>(red + ((warp * kBT + j) * 32 + lane) * NACC + e) =
+            make_float4(acc[j][e], acc[j][e + 1], acc[j][e + 2], acc[j][e + 3]);
+#pragma unroll
+      for (int e = 0; e < NACC; ++e) acc[j][e] = 0.f;
     }
-
-    Buf buf[D];
-#pragma unroll
-    for (int d = 0; d < D; ++d)
-      if (ga + d < gb) load(P, sm, b, ga + d, ga, tb, warp, lane, pol, buf[d]);
-    for (int g0 = ga; g0 < gb; g0 += D) {
-#pragma unroll
-      for (int d = 0; d < D; ++d) {
-        const int g = g0 + d;
-        if (g < gb) {
-          if (warp * T < tb) compute(P, sm, g, tb, warp, lane, buf[d], acc);
-          if constexpr (OUTL) outliers(P, sm, g, ga, buf[d]);
-          if (g + D < gb) load(P, sm, b, g + D, ga, tb, warp, lane, pol, buf[d]);
-        }
-      }
-    }
-
-    // back to the true scale of y
+    consumer_sync(NC * 32);
     float v[T][NACC];
 #pragma unroll
-    for (int i = 0; i < T; ++i)
+    for (int i = 0; i < T; ++i) {
+      const int jj = warp * T + i;
+#pragma unroll
+      for (int e = 0; e < NACC; ++e) v[i][e] = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < NC; ++w2)
+#pragma unroll
+        for (int e = 0; e < NACC; e += 4) {
+          const float4 q =
+              *reinterpret_cast<const float4*>(red + ((w2 * kBT + jj) * 32 + lane) * NACC + e);
+          v[i][e] += q.x;
+          v[i][e + 1] += q.y;
+          v[i][e + 2] += q.z;
+          v[i][e + 3] += q.w;
+        }
 #pragma unroll
       for (int e = 0; e < NACC; ++e)
-        v[i][e] = kLut ? acc[i][e] : acc[i][e] * ((e & 2) ? kTwo24 * Fmt<FMT>::kHiScale : kTwo24);
-
+        if (!kLut) v[i][e] *= (e & 2) ? kTwo24 * Fmt<FMT>::kHiScale : kTwo24;
+    }
     if constexpr (OUTL) {
-      __syncthreads();  // every thread's outliers of the range are in sm.ysm
       const int gi = lane >> 2, t4 = lane & 3;
 #pragma unroll
       for (int i = 0; i < T; ++i) {
@@ -453,23 +504,21 @@ struct Gemv {
           const int m = 2 * t4 + (e & 1) + 8 * (e >> 2);
           const int col = jj * kTileN + gi + ((e & 2) ? 8 : 0);
           if (m < P.M) {
-            v[i][e] += sm.ysm[m][col];
-            sm.ysm[m][col] = 0.f;
+            v[i][e] += ysm[m * 128 + col];
+            ysm[m * 128 + col] = 0.f;
           }
         }
       }
-      __syncthreads();  // cleared before the next range adds into it
     }
-
     if (warp * T >= tb) return;
-    if (ga == 0 && gb == P.G) {  // this CTA owns the whole block
+    if (whole) {
       store_y(P, b, warp, lane, tb, v);
       return;
     }
-    // split-K fix-up
+    // split-K fix-up: publish this CTA's partial, the last contributor sums them all
     const int c = blockIdx.x;
     const int slot = (b == first_block) ? 2 * c : 2 * c + 1;
-    float* dst = P.partials + ((size_t)(slot * W + warp) * T * 32 + lane) * NACC;
+    float* dst = P.partials + ((size_t)(slot * NC + warp) * T * 32 + lane) * NACC;
 #pragma unroll
     for (int i = 0; i < T; ++i)
 #pragma unroll
@@ -479,7 +528,7 @@ struct Gemv {
     __threadfence();
     __syncwarp();
     uint32_t prev = 0;
-    if (lane == 0) prev = atomicAdd(P.counters + (size_t)b * W + warp, 1u);
+    if (lane == 0) prev = atomicAdd(P.counters + (size_t)b * NC + warp, 1u);
     prev = __shfl_sync(0xffffffffu, prev, 0);
     const long long ub = (long long)b * P.G;
     const int cf = cta_of_unit(ub, P.U, P.C);
@@ -493,7 +542,7 @@ struct Gemv {
       for (int e = 0; e < NACC; ++e) s[i][e] = 0.f;
     for (int cc = cf; cc <= cl; ++cc) {
       const int sl = (unit_begin(cc, P.U, P.C) >= ub) ? 2 * cc : 2 * cc + 1;
-      const float* src = P.partials + ((size_t)(sl * W + warp) * T * 32 + lane) * NACC;
+      const float* src = P.partials + ((size_t)(sl * NC + warp) * T * 32 + lane) * NACC;
 #pragma unroll
       for (int i = 0; i < T; ++i)
 #pragma unroll
@@ -506,35 +555,201 @@ struct Gemv {
         }
     }
     store_y(P, b, warp, lane, tb, s);
-    if (lane == 0) P.counters[(size_t)b * W + warp] = 0u;  // ready for the next call
+    if (lane == 0) P.counters[(size_t)b * NC + warp] = 0u;  // ready for the next call
+  }
+
+  // Producer: one lane streams the CTA's units through the ring.
+  __device__ static void produce(const GemvParams& P, uint8_t* smem, long long u0, int n) {
+    const uint32_t ring = smem_addr(smem);
+    const uint32_t bars = ring + C_::kBarOff;
+    const uint64_t pol = evict_first_policy();
+    int b = (int)(u0 / P.G), g = (int)(u0 - (long long)b * P.G);
+    for (int i = 0; i < n; ++i) {
+      const int s = i % S;
+      if (i >= S && !mbar_wait(bars + 8 * (S + s), ((i / S) - 1) & 1))
+        atomicOr(P.err, kErrEmptyTimeout);
+      const int tb = tiles_in_block(b, P.ntiles);
+      const long long ch = chunk_index(b, g, 0, P.G, P.ntiles);
+      const uint32_t st = ring + s * C_::kStageBytes;
+      const uint32_t full = bars + 8 * s;
+      const uint32_t code_bytes = tb * C_::kChunkBytes;
+      const uint32_t param_bytes = tb * C_::kParamChunk;
+      const uint32_t x_bytes = 256u * P.M;
+      mbar_arrive_expect_tx(full, code_bytes + (kLut ? 1 : 2) * param_bytes + x_bytes);
+      bulk_g2s(st, P.qw + ch * C_::kChunkBytes, code_bytes, full, pol);
+      if constexpr (kLut) {
+        bulk_g2s(st + C_::kCodeBytes, static_cast<const float*>(P.zp) + ch * 32, param_bytes, full,
+                 pol);
+      } else {
+        bulk_g2s(st + C_::kCodeBytes, P.sc + ch * 16, param_bytes, full, pol);
+        bulk_g2s(st + C_::kCodeBytes + 256, static_cast<const __half*>(P.zp) + ch * 16,
+                 param_bytes, full, pol);
+      }
+      const __half* xg = P.x + (size_t)g * kGroup;
+      for (int m = 0; m < P.M; ++m)
+        bulk_g2s(st + C_::kXOff + m * C_::kXStride, xg + (size_t)m * P.K, 256u, full);
+      if (++g == P.G) {
+        g = 0;
+        ++b;
+      }
+    }
+  }
+
+  // One unit (block b, group g) of the CTA's range, all its tiles, by one warp.
+  __device__ static void unit(const GemvParams& P, uint8_t* smem, int i, int b, int warp,
+                              int lane, float (&acc)[kBT][NACC], uint32_t (&orc)[3],
+                              uint32_t (&oval)[3], int n) {
+    const uint32_t ring = smem_addr(smem);
+    const uint32_t bars = ring + C_::kBarOff;
+    const uint32_t lut = ring + C_::kLutOff;
+    const int s = i % S;
+    const int tb = tiles_in_block(b, P.ntiles);
+    const uint32_t st = ring + s * C_::kStageBytes;
+    if (!mbar_wait(bars + 8 * s, (i / S) & 1)) atomicOr(P.err, kErrFullTimeout);
+    uint4 xr[4], xr2[4];
+    read_x(P, st, lane, xr, xr2);
+    if constexpr (OUTL) {
+      // outliers of this unit with x from the stage, then prefetch the warp's next unit's
+      float* ysm = reinterpret_cast<float*>(smem + C_::kYsmOff);
+      const uint32_t* toff = reinterpret_cast<const uint32_t*>(smem + C_::kToffOff);
+      const uint32_t e0 = toff[i] + lane, e1 = toff[i + 1];
+      auto add_outlier = [&](uint32_t rc, uint32_t vb) {
+        const int row = rc & 0xFF, col = rc >> 8;
+        const float v = __half2float(__ushort_as_half((unsigned short)vb));
+        const uint32_t xa = st + C_::kXOff + 2 * row;
+        for (int m = 0; m < P.M; ++m) {
+          const float xv = __half2float(__ushort_as_half(lds16(xa + m * C_::kXStride)));
+          atomicAdd(ysm + m * 128 + col, v * xv);
+        }
+      };
+#pragma unroll
+      for (int k = 0; k < 3; ++k)
+        if (e0 + 32 * k < e1) add_outlier(orc[k], oval[k]);
+      for (uint32_t e = e0 + 96; e < e1; e += 32)  // tiles with more than 96 outliers
+        add_outlier(__ldg(P.tile_rc + e), __ldg(P.tile_val + e));
+      prefetch_outliers(P, toff, i + NC, n, lane, orc, oval);
+    }
+    float cx[NACC];
+    if constexpr (kLut) {
+#pragma unroll
+      for (int e = 0; e < NACC; ++e) cx[e] = 0.f;
+    } else {  // sum of x over the group, in the row scales of the codes
+      const uint32_t ones[4] = {kOnesLo, Fmt<FMT>::kOnesHi, kOnesLo, Fmt<FMT>::kOnesHi};
+      hmma0(&cx[0], ones, xr[0].x, xr[0].y);
+      if constexpr (MT == 2) hmma0(&cx[4], ones, xr2[0].x, xr2[0].y);
+#pragma unroll
+      for (int s8 = 1; s8 < 8; ++s8) {
+        const int p = s8 >> 1, h = s8 & 1;
+        hmma(&cx[0], ones, h ? xr[p].z : xr[p].x, h ? xr[p].w : xr[p].y);
+        if constexpr (MT == 2) hmma(&cx[4], ones, h ? xr2[p].z : xr2[p].x, h ? xr2[p].w : xr2[p].y);
+      }
+    }
+    const uint32_t empty = bars + 8 * (S + s);
+    // Tiles 0..3, then 4..7 (of a ragged block some of the second four read stale bytes
+    // whose sums are never written out).  With M <= 8 all eight tiles fit in registers:
+    // the stage is released before any math, so the ring stays in flight.
+    Quad q0, q1;
+    load_quad(st, 0, lane, q0);
+    if constexpr (MT == 1) {
+      if (tb > kQ) load_quad(st, kQ, lane, q1);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty);  // the unit's shared-memory reads are issued
+    } else if (tb <= kQ) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty);
+    }
+    compute_quad(q0, 0, lane, lut, P.mul_shr8, xr, xr2, cx, acc);
+    if (tb > kQ) {
+      if constexpr (MT == 2) {
+        load_quad(st, kQ, lane, q1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty);
+      }
+      compute_quad(q1, kQ, lane, lut, P.mul_shr8, xr, xr2, cx, acc);
+    }
+  }
+
+  __device__ static void prefetch_outliers(const GemvParams& P, const uint32_t* toff, int i, int n,
+                                           int lane, uint32_t (&orc)[3], uint32_t (&oval)[3]) {
+    if (i >= n) return;
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const uint32_t e = toff[i] + lane + 32 * k;
+      if (e < toff[i + 1]) {
+        orc[k] = __ldg(P.tile_rc + e);
+        oval[k] = __ldg(P.tile_val + e);
+      }
+    }
+  }
+
+  // Consumer warp `warp` takes units i = warp, warp + NC, ... of the CTA's range (the
+  // stages i mod S are then private to it), all tiles of each.  At the end of every
+  // run of units of one block the warps meet and combine their sums.
+  __device__ static void consume(const GemvParams& P, uint8_t* smem, long long u0, int n,
+                                 int warp, int lane) {
+    const int first_block = (int)(u0 / P.G);
+    float acc[kBT][NACC];
+#pragma unroll
+    for (int j = 0; j < kBT; ++j)
+#pragma unroll
+      for (int e = 0; e < NACC; ++e) acc[j][e] = 0.f;
+    uint32_t orc[3] = {0, 0, 0}, oval[3] = {0, 0, 0};
+    if constexpr (OUTL)
+      prefetch_outliers(P, reinterpret_cast<const uint32_t*>(smem + C_::kToffOff), warp, n, lane,
+                        orc, oval);
+    int b = first_block, g0 = (int)(u0 - (long long)first_block * P.G);
+    for (int i0 = 0; i0 < n; ++b) {
+      const int len = (n - i0) < (P.G - g0) ? (n - i0) : (P.G - g0);
+      const int i1 = i0 + len;
+      for (int i = i0 + ((warp - i0 % NC) + NC) % NC; i < i1; i += NC)
+        unit(P, smem, i, b, warp, lane, acc, orc, oval, n);
+      finish_block(P, smem, b, g0 == 0 && len == P.G, first_block, warp, lane, acc);
+      i0 = i1;
+      g0 = 0;
+    }
   }
 };
 
-template <int FMT, int MT, int T, int W, int D, bool OUTL>
-__global__ void __launch_bounds__(W * 32) qgemv_kernel(const GemvParams P) {
-  using G_ = Gemv<FMT, MT, T, W, D, OUTL>;
-  __shared__ typename G_::Smem sm;
+template <int FMT, int MT, bool OUTL>
+__global__ void __launch_bounds__(Cfg<FMT, MT, OUTL>::kThreads, 1) qgemv_kernel(const GemvParams P) {
+  using G_ = Gemv<FMT, MT, OUTL>;
+  using C_ = Cfg<FMT, MT, OUTL>;
+  extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if constexpr (G_::kLut) {
-    build_lut_table(sm.lut, P.sc, threadIdx.x, G_::kThreads);
-  }
-  if constexpr (OUTL) {
-    for (int i = threadIdx.x; i < 16 * 128; i += G_::kThreads) (&sm.ysm[0][0])[i] = 0.f;
-  }
-  if constexpr (G_::kLut || OUTL) __syncthreads();
-  const uint64_t pol = evict_first_policy();
   const long long u0 = unit_begin(blockIdx.x, P.U, P.C);
   const long long u1 = unit_begin(blockIdx.x + 1, P.U, P.C);
-  const int first_block = (int)(u0 / P.G);
-  for (long long u = u0; u < u1;) {
-    const int b = (int)(u / P.G);
-    const int ga = (int)(u - (long long)b * P.G);
-    const long long be = (long long)(b + 1) * P.G;
-    const long long ue = u1 < be ? u1 : be;
-    const int gb = ga + (int)(ue - u);
-    G_::segment(P, sm, b, ga, gb, first_block, warp, lane, pol);
-    u = ue;
+  const int n = (int)(u1 - u0);
+  if (threadIdx.x == 0) {
+    const uint32_t bars = smem_addr(smem) + C_::kBarOff;
+    for (int s = 0; s < C_::S; ++s) {
+      mbar_init(bars + 8 * s, 1);            // full: the producer's expect_tx arrival
+      mbar_init(bars + 8 * (C_::S + s), 1);  // empty: the one consumer warp of the stage
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if constexpr (G_::kLut) {
+    build_lut_table(reinterpret_cast<uint32_t*>(smem + C_::kLutOff), P.sc, threadIdx.x,
+                    C_::kThreads);
+  }
+  // x rows M .. kXRows-1 of every stage are never copied: keep them zero
+  for (int e = threadIdx.x; e < C_::S * C_::kXRows * (C_::kXStride / 4); e += C_::kThreads) {
+    const int st = e / (C_::kXRows * (C_::kXStride / 4));
+    const int r = (e / (C_::kXStride / 4)) % C_::kXRows;
+    if (r >= P.M)
+      reinterpret_cast<uint32_t*>(smem + st * C_::kStageBytes + C_::kXOff)[e % (C_::kXRows * (C_::kXStride / 4))] = 0u;
+  }
+  if constexpr (OUTL) {
+    float* ysm = reinterpret_cast<float*>(smem + C_::kYsmOff);
+    for (int i = threadIdx.x; i < 16 * 128; i += C_::kThreads) ysm[i] = 0.f;
+    uint32_t* toff = reinterpret_cast<uint32_t*>(smem + C_::kToffOff);
+    for (int i = threadIdx.x; i <= n; i += C_::kThreads) toff[i] = __ldg(P.tile_off + u0 + i);
+  }
+  __syncthreads();
+  if (warp == C_::NC) {
+    if (lane == 0) G_::produce(P, smem, u0, n);
+    return;
+  }
+  G_::consume(P, smem, u0, n, warp, lane);
 }
 
 }  // namespace qlk

@@ -13,7 +13,12 @@
 // units reads one contiguous byte range.  Only the last block may hold fewer
 // than 8 tiles.
 //
-// Inside a chunk every lane (gi = lane / 4, t = lane % 4) owns the A fragment of
+// Inside a chunk the words of each lane are stored as 16-byte quads: word w of lane
+// l sits at 32-bit index ((w / 4) * 32 + l) * 4 + w % 4, so that one 128-bit access
+// of a whole warp covers 512 contiguous bytes (coalesced in global memory,
+// conflict-free in shared memory).
+//
+// Every lane (gi = lane / 4, t = lane % 4) owns the A fragment of
 // tensor-core step s (s = 0..7, 16 K each): rows gi and gi + 8 of the tile and
 // the K slots {2t, 2t+1, 2t+8, 2t+9}.  The packer maps those slots to the four
 // consecutive k = 128 g + 32 (s / 2) + 8 t + 4 (s % 2) + dk, dk = 0..3, so that
@@ -58,6 +63,9 @@ QL_HD int words_per_lane(int fmt) {
 }
 QL_HD int chunk_bytes(int fmt) { return 128 * words_per_lane(fmt); }
 QL_HD int code_bits(int fmt) { return fmt == kLUT4 ? 4 : fmt; }
+
+// 32-bit index, inside its chunk, of word w of lane l
+QL_HD int word_index(int w, int lane) { return ((w >> 2) * 32 + lane) * 4 + (w & 3); }
 
 QL_HD int tiles_in_block(int b, int ntiles) {
   int r = ntiles - kBlockTiles * b;

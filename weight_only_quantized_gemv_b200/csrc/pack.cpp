@@ -73,7 +73,7 @@ extern "C" ql_status qlinear_pack(int fmt, const void* canonical, void* packed, 
                 code_position(fmt, s, dk, r8, &wi, &bit);
                 words[wi] |= canonical_code(fmt, canonical, N, k, n) << bit;
               }
-          memcpy(chunk + lane * WL, words, sizeof(uint32_t) * WL);
+          for (int w = 0; w < WL; ++w) chunk[word_index(w, lane)] = words[w];
         }
       }
     }

@@ -14,11 +14,8 @@ using namespace qlayout;
 
 namespace {
 
-// Kernel configuration: warps per CTA x tiles per warp = 8 tiles = one 128-column block.
-constexpr int kT = 2;
-constexpr int kW = 4;
-constexpr int kD = 2;
 constexpr int kMaxCtasPerSm = 8;
+constexpr size_t kErrBytes = 256;  // workspace[0..255]: error word (first 4 bytes)
 
 bool fmt_ok(int fmt) { return fmt == kW2 || fmt == kW4 || fmt == kW8 || fmt == kLUT4; }
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
@@ -27,48 +24,54 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 struct Plan {
   int C;            // CTAs
   long long U;      // units
-  int nblocks, ntiles, G, MT;
-  size_t partial_bytes, counter_offset, ws_bytes;
+  int nblocks, ntiles, G, MT, NC, T, threads, smem;
+  size_t counter_offset, partial_offset, ws_bytes;
 };
 
 using KernelPtr = void (*)(qlk::GemvParams);
 
+struct KernelInfo {
+  KernelPtr fn;
+  int threads, smem, NC, T;
+};
+
 template <int FMT, int MT, bool OUTL>
-KernelPtr kernel_ptr() {
-  return qlk::qgemv_kernel<FMT, MT, kT, kW, kD, OUTL>;
+KernelInfo kernel_info() {
+  using C = qlk::Cfg<FMT, MT, OUTL>;
+  return KernelInfo{qlk::qgemv_kernel<FMT, MT, OUTL>, C::kThreads, C::kSmemBytes, C::NC, C::T};
 }
 
-KernelPtr select_kernel(int fmt, int MT, bool outl) {
-  if (outl) return MT == 1 ? kernel_ptr<kW4, 1, true>() : kernel_ptr<kW4, 2, true>();
+KernelInfo select_kernel(int fmt, int MT, bool outl) {
+  if (outl) return MT == 1 ? kernel_info<kW4, 1, true>() : kernel_info<kW4, 2, true>();
   switch (fmt) {
-    case kW2: return MT == 1 ? kernel_ptr<kW2, 1, false>() : kernel_ptr<kW2, 2, false>();
-    case kW4: return MT == 1 ? kernel_ptr<kW4, 1, false>() : kernel_ptr<kW4, 2, false>();
-    case kW8: return MT == 1 ? kernel_ptr<kW8, 1, false>() : kernel_ptr<kW8, 2, false>();
-    default: return MT == 1 ? kernel_ptr<kLUT4, 1, false>() : kernel_ptr<kLUT4, 2, false>();
+    case kW2: return MT == 1 ? kernel_info<kW2, 1, false>() : kernel_info<kW2, 2, false>();
+    case kW4: return MT == 1 ? kernel_info<kW4, 1, false>() : kernel_info<kW4, 2, false>();
+    case kW8: return MT == 1 ? kernel_info<kW8, 1, false>() : kernel_info<kW8, 2, false>();
+    default: return MT == 1 ? kernel_info<kLUT4, 1, false>() : kernel_info<kLUT4, 2, false>();
   }
 }
 
-// Resident CTAs per SM of a kernel on a device (queried once, then cached).
-cudaError_t ctas_per_sm(KernelPtr k, int dev, int* out) {
+// Opt a kernel into its dynamic shared memory and query its resident CTAs per SM
+// (once per kernel and device, then cached).
+cudaError_t prepare_kernel(const KernelInfo& k, int dev, int* ctas) {
   static std::mutex mu;
   static std::unordered_map<uint64_t, int> cache;
-  const uint64_t key = ((uint64_t)(uintptr_t)k << 8) ^ (uint64_t)dev;
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    auto it = cache.find(key);
-    if (it != cache.end()) {
-      *out = it->second;
-      return cudaSuccess;
-    }
+  const uint64_t key = ((uint64_t)(uintptr_t)k.fn << 8) ^ (uint64_t)dev;
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) {
+    *ctas = it->second;
+    return cudaSuccess;
   }
+  cudaError_t e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
+  if (e != cudaSuccess) return e;
   int occ = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kW * 32, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k.fn, k.threads, k.smem);
   if (e != cudaSuccess) return e;
   if (occ < 1) occ = 1;
   if (occ > kMaxCtasPerSm) occ = kMaxCtasPerSm;
-  std::lock_guard<std::mutex> lk(mu);
   cache[key] = occ;
-  *out = occ;
+  *ctas = occ;
   return cudaSuccess;
 }
 
@@ -80,9 +83,14 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   p->MT = M <= 8 ? 1 : 2;
+  const KernelInfo k = select_kernel(fmt, p->MT, outl);
   int occ = 1;
-  e = ctas_per_sm(select_kernel(fmt, p->MT, outl), dev, &occ);
+  e = prepare_kernel(k, dev, &occ);
   if (e != cudaSuccess) return e;
+  p->NC = k.NC;
+  p->T = k.T;
+  p->threads = k.threads;
+  p->smem = k.smem;
   p->G = K / kGroup;
   p->ntiles = N / kTileN;
   p->nblocks = (p->ntiles + kBlockTiles - 1) / kBlockTiles;
@@ -93,11 +101,16 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
     const long long v = atoll(cap);
     if (v > 0 && v < C) C = v;
   }
+  if (outl) {  // a CTA keeps the Tile-COO offsets of its units in shared memory
+    const long long cmin = (p->U + qlk::kMaxUnitsPerCta - 1) / qlk::kMaxUnitsPerCta;
+    if (C < cmin) C = cmin;
+  }
   if (C > p->U) C = p->U;
   p->C = (int)C;
-  p->partial_bytes = (size_t)2 * p->C * kW * kT * 32 * 4 * p->MT * sizeof(float);
-  p->counter_offset = align_up(p->partial_bytes, 256);
-  p->ws_bytes = p->counter_offset + align_up((size_t)p->nblocks * kW * sizeof(uint32_t), 256);
+  p->counter_offset = kErrBytes;
+  p->partial_offset = align_up(p->counter_offset + (size_t)p->nblocks * p->NC * sizeof(uint32_t), 256);
+  p->ws_bytes = p->partial_offset +
+                (size_t)2 * p->C * p->NC * p->T * 32 * 4 * p->MT * sizeof(float);
   return cudaSuccess;
 }
 
@@ -126,7 +139,7 @@ ql_status run(const Call& c) {
   if (!c.x || !c.qw || !c.p0 || !c.p1 || !c.y) return QL_ERR_NULL;
   if (c.outl && (!c.toff || !c.trc || !c.tval)) return QL_ERR_NULL;
   if (!shape_ok(c.M, c.N, c.K)) return QL_ERR_SHAPE;
-  if (c.outl && (c.N % 128 || c.K / kGroup > qlk::kMaxOutlierGroups)) return QL_ERR_SHAPE;
+  if (c.outl && c.N % 128) return QL_ERR_SHAPE;
   if (!aligned(c.x, 16) || !aligned(c.qw, 32) || !aligned(c.y, 2)) return QL_ERR_ALIGN;
   if (c.fmt == kLUT4) {
     if (!aligned(c.p0, 2) || !aligned(c.p1, 16)) return QL_ERR_ALIGN;
@@ -148,8 +161,9 @@ ql_status run(const Call& c) {
   P.tile_rc = reinterpret_cast<const uint16_t*>(c.trc);
   P.tile_val = c.tval;
   P.y = static_cast<__half*>(c.y);
-  P.partials = static_cast<float*>(c.ws);
+  P.err = static_cast<uint32_t*>(c.ws);
   P.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(c.ws) + p.counter_offset);
+  P.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(c.ws) + p.partial_offset);
   P.M = c.M;
   P.N = c.N;
   P.K = c.K;
@@ -158,8 +172,9 @@ ql_status run(const Call& c) {
   P.ntiles = p.ntiles;
   P.U = p.U;
   P.C = p.C;
-  KernelPtr k = select_kernel(c.fmt, p.MT, c.outl);
-  k<<<p.C, kW * 32, 0, c.stream>>>(P);
+  P.mul_shr8 = 1u << 24;
+  const KernelInfo k = select_kernel(c.fmt, p.MT, c.outl);
+  k.fn<<<p.C, k.threads, k.smem, c.stream>>>(P);
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
@@ -191,9 +206,9 @@ __global__ void __launch_bounds__(128) debug_kernel(const uint8_t* packed, const
   const long long ch = chunk_index(b, g, jj, G, ntiles);
   constexpr int KW = qlk::Fmt<FMT>::kWords;
   uint32_t wv[KW];
-  const uint32_t* src = reinterpret_cast<const uint32_t*>(packed + ch * chunk_bytes(FMT)) + lane * KW;
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(packed + ch * chunk_bytes(FMT));
 #pragma unroll
-  for (int i = 0; i < KW; ++i) wv[i] = src[i];
+  for (int i = 0; i < KW; ++i) wv[i] = src[word_index(i, lane)];
   const int gi = lane >> 2, t4 = lane & 3;
   float2 s2 = make_float2(0.f, 0.f), z2 = s2;
   float4 am = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -209,10 +224,10 @@ __global__ void __launch_bounds__(128) debug_kernel(const uint8_t* packed, const
   for (int s = 0; s < 8; ++s) {
     uint32_t a[4];
     if constexpr (FMT == kLUT4) {
-      if (DEQ) qlk::frag_lut(wv[s], tbl, lane, a);
+      if (DEQ) qlk::frag_lut(wv[s], (uint32_t)__cvta_generic_to_shared(tbl), lane, a);
       else a[0] = a[1] = a[2] = a[3] = 0u;
     } else {
-      qlk::frag_uniform<FMT>(wv, s, a);
+      qlk::frag_uniform<FMT>(wv, s, 1u << 24, a);
     }
 #pragma unroll
     for (int r = 0; r < 4; ++r)
@@ -298,8 +313,8 @@ extern "C" ql_status qlinear_plan(int fmt, int M, int N, int K, ql_plan* plan) {
   Plan p;
   if (make_plan(fmt, M, N, K, false, &p) != cudaSuccess) return QL_ERR_CUDA;
   plan->ctas = p.C;
-  plan->warps = kW;
-  plan->tiles_per_warp = kT;
+  plan->warps = p.NC;
+  plan->tiles_per_warp = p.T;
   plan->units = p.U;
   plan->m_bucket = p.MT;
   return QL_OK;
@@ -360,4 +375,13 @@ extern "C" ql_status qlinear_debug_dequant(int fmt, const void* packed, const vo
   if (fmt == kLUT4 ? !aligned(p1, 16) : (!aligned(p0, 4) || !aligned(p1, 4))) return QL_ERR_ALIGN;
   return launch_debug<true>(fmt, packed, p0, p1, nullptr, w, N, K,
                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" ql_status qlinear_read_error(void* workspace, uint32_t* flags, ql_stream_t stream) {
+  if (!workspace || !flags) return QL_ERR_NULL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(flags, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return QL_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), st) != cudaSuccess) return QL_ERR_CUDA;
+  return cudaStreamSynchronize(st) == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
