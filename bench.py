@@ -1,0 +1,459 @@
+"""Benchmark of the weight-only-quantized GEMV on B200.
+
+One step = one pass of the hot path over the six Llama-shaped W4A16 g128 decode
+layers at M = 1: (K, N) = (4096, 12288), (4096, 4096), (4096, 28672), (14336, 4096),
+(8192, 28672), (28672, 8192), each a separate call of qlinear_w4a16 on its own
+resident packed weights (379 MB in total, cycled every step, so no layer is
+L2-resident when it is read again).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line.  `value` is the achieved algorithmic bandwidth of the whole
+job (packed codes + scales/zeros + x + y bytes of every layer of every step on every
+rank, divided by the slowest rank's device time).  `--impl reference` times the CPU
+oracle on a bounded sample of the same workload instead.  Under torchrun every rank
+runs an independent replica (the layer does not shard across GPUs in this workload).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import platform
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A16-g128 dequant-GEMV µs/layer at M=1; achieved HBM GB/s vs B200 peak"
+SHAPES = [(4096, 12288), (4096, 4096), (4096, 28672), (14336, 4096), (8192, 28672), (28672, 8192)]
+WORKLOAD = 1  # seeds 1000 * workload + layer
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["weight_only_quantized_gemv_b200/csrc/kernels.cuh",
+                  "weight_only_quantized_gemv_b200/csrc/layout.h",
+                  "weight_only_quantized_gemv_b200/csrc/qlinear.cu"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "qgemv_w4_llama_m1_traffic.txt")
+
+
+def algorithmic_bytes(K, N, M=1):
+    """Packed codes + fp16 scales and zeros + fp16 x + fp16 y, each counted once."""
+    return K * N // 2 + 2 * (K // 128) * N * 2 + M * K * 2 + M * N * 2
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic():
+    """Per-layer DRAM bytes from the committed ncu summary, if taken on this kernel source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    kv = {}
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    try:
+        return {tuple(int(t) for t in k[len("traffic_bytes_"):].split("x")): float(v)
+                for k, v in kv.items() if k.startswith("traffic_bytes_")}
+    except ValueError:
+        return None
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas)
+
+
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    return rank, world, local
+
+
+def init_pg(local, world):
+    if world == 1:
+        return None
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return dist
+
+
+# ---------------------------------------------------------------------------
+
+
+def cpu_oracle_sample(layers, seconds=10.0, cols=64):
+    """Time the fp64 oracle on column slices of the six layers, single-threaded BLAS.
+
+    `layers`: (UniformLayer, x, K, N) of the benchmarked workload."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(1)
+    except ImportError:
+        limiter = None
+    done_bytes = 0.0
+    t0 = time.perf_counter()
+    rounds = 0
+    rs = np.random.default_rng(0)
+    while time.perf_counter() - t0 < seconds:
+        for u, x, K, N in layers:
+            c = rs.choice(N, size=cols, replace=False)
+            oracle.gemv_uniform(x, u.qweight, u.scales, u.zeros, 4, 128, cols=c)
+            done_bytes += algorithmic_bytes(K, cols)
+        rounds += 1
+    el = time.perf_counter() - t0
+    if limiter is not None:
+        limiter.unregister()
+    return {"value": done_bytes / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rounds} rounds of {cols} random columns of each of the six layers "
+                      f"(fp64 unpack + eager dequant + dot), {el:.1f} s",
+            "cpu": platform.processor() or platform.machine(),
+            "host_cores": len(os.sched_getaffinity(0))}
+
+
+def run_reference(args):
+    rank, world, local = dist_setup(args.gpus)
+    if rank != 0:
+        return
+    # the oracle on the host cores: each step is a bounded sample of the workload
+    import oracle
+    from synth import gen
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+    except ImportError:
+        pass
+    cols = args.ref_cols
+    layers = []
+    for j, (K, N) in enumerate(SHAPES):
+        seed = gen.workload_seed(WORKLOAD, j)
+        u = gen.uniform_layer(seed, K, N, 4)
+        x = gen.activations(seed, 1, K)
+        layers.append((u, x, K, N))
+    rs = np.random.default_rng(1)
+
+    def step():
+        b = 0
+        for u, x, K, N in layers:
+            c = rs.choice(N, size=cols, replace=False)
+            oracle.gemv_uniform(x, u.qweight, u.scales, u.zeros, 4, 128, cols=c)
+            b += algorithmic_bytes(K, cols)
+        return b
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    total = 0
+    for _ in range(args.steps):
+        total += step()
+    el = time.perf_counter() - t0
+    value = total / el / 1e9
+    sample = f"{cols} random columns of each of the six layers per step (fp64 unpack + eager dequant + dot)"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "W4A16 g128 M=1, six Llama-shaped decode layers (CPU oracle sample)",
+                   "layers": [list(s) for s in SHAPES], "M": 1, "columns_per_layer": cols},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def run_gpu(args):
+    import torch
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dist = init_pg(local, world)
+    dev = torch.device("cuda", local)
+    from synth import gen
+    from weight_only_quantized_gemv_b200 import layers as qlayers
+    import weight_only_quantized_gemv_b200 as ql
+
+    lays, xs, ys, byts, host_layers = [], [], [], [], []
+    for j, (K, N) in enumerate(SHAPES):
+        seed = gen.workload_seed(WORKLOAD, j)
+        u = gen.uniform_layer(seed, K, N, 4)
+        lays.append(qlayers.from_uniform(u, dev, max_m=1))
+        x = gen.activations(seed, 1, K)
+        xs.append(torch.from_numpy(x).to(dev))
+        ys.append(torch.empty((1, N), dtype=torch.float16, device=dev))
+        byts.append(algorithmic_bytes(K, N))
+        u.codes = None  # the oracle reads the canonical packed words
+        host_layers.append((u, x, K, N))
+    step_bytes = float(sum(byts))
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+
+    def eager_step():
+        for j, lay in enumerate(lays):
+            lay.forward(xs[j], ys[j], stream)
+
+    # warm-up outside any graph (the library's one-time per-kernel set-up happens here)
+    for _ in range(3):
+        eager_step()
+    torch.cuda.synchronize()
+
+    def capture(nsteps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(nsteps):
+                eager_step()
+        return g
+    # The timed region replays graphs of whole steps, so the host never gates the device:
+    # one graph holds 10 steps (60 launches), a one-step graph covers the remainder.
+    g10, g1 = capture(10), capture(1)
+    torch.cuda.synchronize()
+
+    def steps(n):
+        for _ in range(n // 10):
+            g10.replay()
+        for _ in range(n % 10):
+            g1.replay()
+
+    steps(args.warmup)
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        steps(args.steps)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms = start.elapsed_time(stop)
+    err = max(ql.qlinear_read_error(lay.workspace) for lay in lays)
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    del g10, g1
+
+    # per-layer breakdown: 30 launches of one layer over three copies of its packed weights
+    # (so none is L2-resident), one graph, CUDA events around 10 replays
+    per_layer_us = []
+    for j, lay in enumerate(lays):
+        copies = [lay.qweight, lay.qweight.clone(), lay.qweight.clone()]
+        pscale = [lay.p0, lay.p0.clone(), lay.p0.clone()]
+        pzero = [lay.p1, lay.p1.clone(), lay.p1.clone()]
+        orig = (lay.qweight, lay.p0, lay.p1)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for r in range(30):
+                lay.qweight, lay.p0, lay.p1 = copies[r % 3], pscale[r % 3], pzero[r % 3]
+                lay.forward(xs[j], ys[j], stream)
+        lay.qweight, lay.p0, lay.p1 = orig
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(10):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        per_layer_us.append(e0.elapsed_time(e1) * 1e3 / 300)
+        del g, copies, pscale, pzero
+    per_layer_ms = np.array(per_layer_us) / 1e3
+
+    # end to end through the public API: x host->device, the call, y device->host
+    hx = [torch.empty_like(x, device="cpu").pin_memory().copy_(x.cpu()) for x in xs]
+    hy = [torch.empty_like(y, device="cpu").pin_memory() for y in ys]
+    e2e_steps = max(3, min(args.steps, 200))
+
+    def e2e_step():
+        for j, lay in enumerate(lays):
+            xs[j].copy_(hx[j], non_blocking=True)
+            lay.forward(xs[j], ys[j], stream)
+            hy[j].copy_(ys[j], non_blocking=True)
+        stream.synchronize()
+    for _ in range(2):
+        e2e_step()
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    if rank == 0:
+        peak, peak_src = measured_peaks()
+        # every launch in the timed region is the GEMV kernel: its average launch duration is
+        # the region's device time over the launches, bytes per launch the step's over six
+        launch_ms = ms / args.steps
+        achieved = step_bytes / (launch_ms * 1e-3) / 1e9
+        traffic = read_traffic()
+        traffic_per_launch = None
+        if traffic is not None and all(s in traffic for s in SHAPES):
+            traffic_per_launch = float(np.mean([traffic[s] for s in SHAPES]))
+        layers_out = []
+        for (K, N), b, t in zip(SHAPES, byts, per_layer_ms):
+            layers_out.append({"K": K, "N": N, "us": round(t * 1e3, 3), "bytes": b,
+                               "GBs": round(b / (t * 1e-3) / 1e9, 1),
+                               "frac": round(b / (t * 1e-3) / 1e9 / peak, 4)})
+        clocks = clk.summary()
+        out = {
+            "metric": METRIC,
+            "value": step_bytes * world / (ms * 1e-3 / args.steps) / 1e9,
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms / args.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f16",
+            "data": "synthetic",
+            "config": {
+                "workload": "W4A16 asymmetric g128 GEMV, M=1, six Llama-shaped decode layers",
+                "layers": [list(s) for s in SHAPES], "M": 1, "group": 128,
+                "l2": "inputs larger than L2: 379 MB of packed weights cycled every step",
+                "parallelism": f"replicas x{world}",
+                "us_per_layer": round(ms * 1e3 / args.steps / len(SHAPES), 3),
+            },
+            "layers": layers_out,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic_per_launch,
+                         "peak_source": peak_src,
+                         "kernel": "qgemv_kernel<W4, M<=8> (one launch per layer)",
+                         "timing": "CUDA events around the timed region (graph replays of whole steps); "
+                                   "the per-layer table comes from a separate 30-launch pass per layer"},
+            "e2e": {"value": step_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": int(sum(x.numel() * 2 for x in xs)),
+                    "d2h_bytes_per_step": int(sum(y.numel() * 2 for y in ys)),
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps * len(SHAPES),
+            "clocks": clocks,
+            "error_flags": err,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            out["cpu_baseline"] = cpu_oracle_sample(host_layers, seconds=args.cpu_seconds)
+        print(json.dumps(out))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--ref-cols", type=int, default=16)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -68,7 +68,7 @@ struct GemvParams {
   uint32_t* counters;         // [nblocks][NC]
   uint32_t* err;              // sticky error flags
   int M, N, K, G, nblocks, ntiles;
-  long long U;                // nblocks * G
+  int U;                      // nblocks * G
   int C;                      // CTAs
   uint32_t mul_shr8;          // 2^24: v >> 8 as mul.hi on the FMA pipe (set by the host)
 };
@@ -78,25 +78,25 @@ template <> struct Fmt<kW4> {
   static constexpr int kWords = 8;
   static constexpr uint32_t kOnesHi = 0x00100010u;  // rows gi+8 carry a factor 16
   static constexpr float kHiScale = 1.0f / 16.0f;
-  static constexpr int kStages = 8;
+  static constexpr int kStagesPerWarpM8 = 1;
 };
 template <> struct Fmt<kW2> {
   static constexpr int kWords = 4;
   static constexpr uint32_t kOnesHi = 0x00040004u;  // rows gi+8 carry a factor 4
   static constexpr float kHiScale = 1.0f / 4.0f;
-  static constexpr int kStages = 12;
+  static constexpr int kStagesPerWarpM8 = 2;
 };
 template <> struct Fmt<kW8> {
   static constexpr int kWords = 16;
   static constexpr uint32_t kOnesHi = 0x00010001u;
   static constexpr float kHiScale = 1.0f;
-  static constexpr int kStages = 8;
+  static constexpr int kStagesPerWarpM8 = 1;
 };
 template <> struct Fmt<kLUT4> {
   static constexpr int kWords = 8;
   static constexpr uint32_t kOnesHi = 0;
   static constexpr float kHiScale = 1.0f;
-  static constexpr int kStages = 8;
+  static constexpr int kStagesPerWarpM8 = 1;
 };
 
 constexpr uint32_t kOnesLo = 0x00010001u;  // fp16 pair (2^-24, 2^-24)
@@ -112,8 +112,9 @@ struct Cfg {
   static constexpr int kThreads = (NC + 1) * 32;     // + one producer warp
   static constexpr int KW = Fmt<FMT>::kWords;
   static constexpr int NACC = 4 * MT;
-  static constexpr int S = Fmt<FMT>::kStages;        // a multiple of NC: warp w uses stages w mod NC
-  static_assert(S % NC == 0, "stages must split evenly over the consumer warps");
+  // stages: a multiple of NC, warp w uses the stages s = w (mod NC)
+  static constexpr int S = NC * (MT == 1 ? Fmt<FMT>::kStagesPerWarpM8 : 2);
+  static constexpr int kMinCtas = (MT == 1 && FMT != kW8 && FMT != kLUT4) ? 3 : 1;
   static constexpr int kChunkBytes = 128 * KW;
   static constexpr int kCodeBytes = kBlockTiles * kChunkBytes;
   static constexpr int kParamChunk = (FMT == kLUT4) ? 128 : 32;   // per tile, per array
@@ -286,12 +287,13 @@ __device__ __forceinline__ void build_lut_table(uint32_t* tbl, const __half* lut
 // ---------------------------------------------------------------------------
 // stream-K partition helpers
 
-__host__ __device__ __forceinline__ long long unit_begin(long long c, long long U, long long C) {
-  return c * U / C;
+// 32-bit arithmetic: the host guarantees U * C < 2^31.
+__host__ __device__ __forceinline__ int unit_begin(int c, int U, int C) {
+  return (int)((unsigned)c * (unsigned)U / (unsigned)C);
 }
 // CTA whose unit range contains unit u.
-__host__ __device__ __forceinline__ int cta_of_unit(long long u, long long U, long long C) {
-  return (int)(((u + 1) * C - 1) / U);
+__host__ __device__ __forceinline__ int cta_of_unit(int u, int U, int C) {
+  return (int)(((unsigned)(u + 1) * (unsigned)C - 1u) / (unsigned)U);
 }
 
 // ---------------------------------------------------------------------------
@@ -530,7 +532,7 @@ struct Gemv {
     uint32_t prev = 0;
     if (lane == 0) prev = atomicAdd(P.counters + (size_t)b * NC + warp, 1u);
     prev = __shfl_sync(0xffffffffu, prev, 0);
-    const long long ub = (long long)b * P.G;
+    const int ub = b * P.G;
     const int cf = cta_of_unit(ub, P.U, P.C);
     const int cl = cta_of_unit(ub + P.G - 1, P.U, P.C);
     if (prev + 1 != (uint32_t)(cl - cf + 1)) return;
@@ -540,30 +542,48 @@ struct Gemv {
     for (int i = 0; i < T; ++i)
 #pragma unroll
       for (int e = 0; e < NACC; ++e) s[i][e] = 0.f;
-    for (int cc = cf; cc <= cl; ++cc) {
-      const int sl = (unit_begin(cc, P.U, P.C) >= ub) ? 2 * cc : 2 * cc + 1;
-      const float* src = P.partials + ((size_t)(sl * NC + warp) * T * 32 + lane) * NACC;
+    // contributors in CTA order; loads of up to kF slots are in flight at once
+    constexpr int kF = 4;
+    for (int c0 = cf; c0 <= cl; c0 += kF) {
+      float4 q[kF][T][NACC / 4];
 #pragma unroll
-      for (int i = 0; i < T; ++i)
+      for (int f = 0; f < kF; ++f) {
+        const int cc = c0 + f;
+        if (cc <= cl) {
+          const int sl = (unit_begin(cc, P.U, P.C) >= ub) ? 2 * cc : 2 * cc + 1;
+          const float* src = P.partials + ((size_t)(sl * NC + warp) * T * 32 + lane) * NACC;
 #pragma unroll
-        for (int e = 0; e < NACC; e += 4) {
-          const float4 q = __ldcg(reinterpret_cast<const float4*>(src + (size_t)i * 32 * NACC + e));
-          s[i][e] += q.x;
-          s[i][e + 1] += q.y;
-          s[i][e + 2] += q.z;
-          s[i][e + 3] += q.w;
+          for (int i = 0; i < T; ++i)
+#pragma unroll
+            for (int e = 0; e < NACC; e += 4)
+              q[f][i][e / 4] = __ldcg(reinterpret_cast<const float4*>(src + (size_t)i * 32 * NACC + e));
         }
+      }
+#pragma unroll
+      for (int f = 0; f < kF; ++f) {
+        if (c0 + f <= cl) {
+#pragma unroll
+          for (int i = 0; i < T; ++i)
+#pragma unroll
+            for (int e = 0; e < NACC; e += 4) {
+              s[i][e] += q[f][i][e / 4].x;
+              s[i][e + 1] += q[f][i][e / 4].y;
+              s[i][e + 2] += q[f][i][e / 4].z;
+              s[i][e + 3] += q[f][i][e / 4].w;
+            }
+        }
+      }
     }
     store_y(P, b, warp, lane, tb, s);
     if (lane == 0) P.counters[(size_t)b * NC + warp] = 0u;  // ready for the next call
   }
 
   // Producer: one lane streams the CTA's units through the ring.
-  __device__ static void produce(const GemvParams& P, uint8_t* smem, long long u0, int n) {
+  __device__ static void produce(const GemvParams& P, uint8_t* smem, int u0, int n) {
     const uint32_t ring = smem_addr(smem);
     const uint32_t bars = ring + C_::kBarOff;
     const uint64_t pol = evict_first_policy();
-    int b = (int)(u0 / P.G), g = (int)(u0 - (long long)b * P.G);
+    int b = u0 / P.G, g = u0 - b * P.G;
     for (int i = 0; i < n; ++i) {
       const int s = i % S;
       if (i >= S && !mbar_wait(bars + 8 * (S + s), ((i / S) - 1) & 1))
@@ -648,23 +668,23 @@ struct Gemv {
     // Tiles 0..3, then 4..7 (of a ragged block some of the second four read stale bytes
     // whose sums are never written out).  With M <= 8 all eight tiles fit in registers:
     // the stage is released before any math, so the ring stays in flight.
-    Quad q0, q1;
-    load_quad(st, 0, lane, q0);
-    if constexpr (MT == 1) {
-      if (tb > kQ) load_quad(st, kQ, lane, q1);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty);  // the unit's shared-memory reads are issued
-    } else if (tb <= kQ) {
+    // Tiles 0..3, then 4..7 (of a ragged block some of the second four read stale bytes
+    // whose sums are never written out).  The stage is released once the second
+    // four are in registers, so its refill overlaps their math.
+    {
+      Quad q0;
+      load_quad(st, 0, lane, q0);
+      if (tb <= kQ) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty);  // the unit's last shared-memory reads are issued
+      }
+      compute_quad(q0, 0, lane, lut, P.mul_shr8, xr, xr2, cx, acc);
+    }
+    if (tb > kQ) {
+      Quad q1;
+      load_quad(st, kQ, lane, q1);
       __syncwarp();
       if (lane == 0) mbar_arrive(empty);
-    }
-    compute_quad(q0, 0, lane, lut, P.mul_shr8, xr, xr2, cx, acc);
-    if (tb > kQ) {
-      if constexpr (MT == 2) {
-        load_quad(st, kQ, lane, q1);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty);
-      }
       compute_quad(q1, kQ, lane, lut, P.mul_shr8, xr, xr2, cx, acc);
     }
   }
@@ -685,9 +705,9 @@ struct Gemv {
   // Consumer warp `warp` takes units i = warp, warp + NC, ... of the CTA's range (the
   // stages i mod S are then private to it), all tiles of each.  At the end of every
   // run of units of one block the warps meet and combine their sums.
-  __device__ static void consume(const GemvParams& P, uint8_t* smem, long long u0, int n,
+  __device__ static void consume(const GemvParams& P, uint8_t* smem, int u0, int n,
                                  int warp, int lane) {
-    const int first_block = (int)(u0 / P.G);
+    const int first_block = u0 / P.G;
     float acc[kBT][NACC];
 #pragma unroll
     for (int j = 0; j < kBT; ++j)
@@ -697,7 +717,7 @@ struct Gemv {
     if constexpr (OUTL)
       prefetch_outliers(P, reinterpret_cast<const uint32_t*>(smem + C_::kToffOff), warp, n, lane,
                         orc, oval);
-    int b = first_block, g0 = (int)(u0 - (long long)first_block * P.G);
+    int b = first_block, g0 = u0 - first_block * P.G;
     for (int i0 = 0; i0 < n; ++b) {
       const int len = (n - i0) < (P.G - g0) ? (n - i0) : (P.G - g0);
       const int i1 = i0 + len;
@@ -711,14 +731,15 @@ struct Gemv {
 };
 
 template <int FMT, int MT, bool OUTL>
-__global__ void __launch_bounds__(Cfg<FMT, MT, OUTL>::kThreads, 1) qgemv_kernel(const GemvParams P) {
+__global__ void __launch_bounds__(Cfg<FMT, MT, OUTL>::kThreads, Cfg<FMT, MT, OUTL>::kMinCtas)
+    qgemv_kernel(const GemvParams P) {
   using G_ = Gemv<FMT, MT, OUTL>;
   using C_ = Cfg<FMT, MT, OUTL>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const long long u0 = unit_begin(blockIdx.x, P.U, P.C);
-  const long long u1 = unit_begin(blockIdx.x + 1, P.U, P.C);
-  const int n = (int)(u1 - u0);
+  const int u0 = unit_begin(blockIdx.x, P.U, P.C);
+  const int u1 = unit_begin(blockIdx.x + 1, P.U, P.C);
+  const int n = u1 - u0;
   if (threadIdx.x == 0) {
     const uint32_t bars = smem_addr(smem) + C_::kBarOff;
     for (int s = 0; s < C_::S; ++s) {
@@ -732,11 +753,14 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, OUTL>::kThreads, 1) qgemv_kernel(
                     C_::kThreads);
   }
   // x rows M .. kXRows-1 of every stage are never copied: keep them zero
-  for (int e = threadIdx.x; e < C_::S * C_::kXRows * (C_::kXStride / 4); e += C_::kThreads) {
-    const int st = e / (C_::kXRows * (C_::kXStride / 4));
-    const int r = (e / (C_::kXStride / 4)) % C_::kXRows;
-    if (r >= P.M)
-      reinterpret_cast<uint32_t*>(smem + st * C_::kStageBytes + C_::kXOff)[e % (C_::kXRows * (C_::kXStride / 4))] = 0u;
+  {
+    constexpr int kRowWords = C_::kXStride / 4;
+    const int zrows = C_::kXRows > P.M ? C_::kXRows - P.M : 0;
+    const int per_stage = zrows * kRowWords;
+    for (int e = threadIdx.x; e < C_::S * per_stage; e += C_::kThreads) {
+      const int st = e / per_stage, r = e - st * per_stage;
+      reinterpret_cast<uint32_t*>(smem + st * C_::kStageBytes + C_::kXOff + P.M * C_::kXStride)[r] = 0u;
+    }
   }
   if constexpr (OUTL) {
     float* ysm = reinterpret_cast<float*>(smem + C_::kYsmOff);

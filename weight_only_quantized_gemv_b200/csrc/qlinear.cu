@@ -106,6 +106,8 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
     if (C < cmin) C = cmin;
   }
   if (C > p->U) C = p->U;
+  // the kernel's stream-K index arithmetic is 32-bit
+  if (p->U * C >= (1LL << 31)) return cudaErrorInvalidValue;
   p->C = (int)C;
   p->counter_offset = kErrBytes;
   p->partial_offset = align_up(p->counter_offset + (size_t)p->nblocks * p->NC * sizeof(uint32_t), 256);
@@ -170,7 +172,7 @@ ql_status run(const Call& c) {
   P.G = p.G;
   P.nblocks = p.nblocks;
   P.ntiles = p.ntiles;
-  P.U = p.U;
+  P.U = (int)p.U;
   P.C = p.C;
   P.mul_shr8 = 1u << 24;
   const KernelInfo k = select_kernel(c.fmt, p.MT, c.outl);

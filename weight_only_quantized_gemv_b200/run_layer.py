@@ -1,0 +1,98 @@
+"""Run one quantized-GEMV configuration repeatedly (for timing and profiler captures).
+
+    python -m weight_only_quantized_gemv_b200.run_layer --fmt w4 --K 8192 --N 28672 --M 1 \
+        --launches 4 [--copies 3] [--time]
+
+The packed codes and parameters are random bytes of the right sizes (the kernel's
+speed does not depend on their values), allocated in `--copies` copies that the
+launches cycle through so that no launch finds its weights in L2.  With `--time` the
+launches are replayed from a CUDA graph and the mean device time per launch is
+printed as JSON.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import torch
+
+from . import (FORMATS, QL_FMT_LUT4, qlinear_lut4, qlinear_plan, qlinear_read_error,
+               qlinear_w2a16, qlinear_w4a16, qlinear_w8a16, qlinear_workspace_bytes)
+
+_UNIFORM = {2: qlinear_w2a16, 4: qlinear_w4a16, 8: qlinear_w8a16}
+
+
+def algorithmic_bytes(fmt: int, K: int, N: int, M: int) -> int:
+    if fmt == QL_FMT_LUT4:
+        return K * N // 2 + (K // 64) * N * 4 + 32 + M * K * 2 + M * N * 2
+    return K * N * fmt // 8 + 2 * (K // 128) * N * 2 + M * K * 2 + M * N * 2
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--fmt", choices=sorted(FORMATS), default="w4")
+    ap.add_argument("--K", type=int, default=8192)
+    ap.add_argument("--N", type=int, default=28672)
+    ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--launches", type=int, default=4)
+    ap.add_argument("--copies", type=int, default=3)
+    ap.add_argument("--time", action="store_true")
+    a = ap.parse_args()
+    fmt, K, N, M = FORMATS[a.fmt], a.K, a.N, a.M
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    bits = 4 if fmt == QL_FMT_LUT4 else fmt
+    G = K // 128
+    gen = torch.Generator(device=dev).manual_seed(0)
+    q = [torch.randint(0, 256, (K * N * bits // 8,), dtype=torch.uint8, device=dev, generator=gen)
+         for _ in range(a.copies)]
+    if fmt == QL_FMT_LUT4:
+        p0 = [torch.linspace(-1, 1, 16, device=dev).half().view(torch.int16)] * a.copies
+        p1 = [torch.rand((K // 64) * N, device=dev, generator=gen) * 0.05 for _ in range(a.copies)]
+    else:
+        p0 = [(torch.rand(G * N, device=dev, generator=gen) * 0.01).half().view(torch.int16)
+              for _ in range(a.copies)]
+        p1 = [torch.randint(0, 1 << bits, (G * N,), device=dev, generator=gen).half().view(torch.int16)
+              for _ in range(a.copies)]
+    x = torch.randn(M, K, device=dev, generator=gen).half().view(torch.int16)
+    y = torch.empty(M, N, device=dev, dtype=torch.int16)
+    ws = torch.zeros(qlinear_workspace_bytes(fmt, M, N, K) // 4 + 64, dtype=torch.int32, device=dev)
+    def call(i):  # on the current stream (the capture stream inside the graph below)
+        c = i % a.copies
+        if fmt == QL_FMT_LUT4:
+            qlinear_lut4(x, q[c], p0[c], p1[c], y, M, N, K, ws)
+        else:
+            _UNIFORM[fmt](x, q[c], p0[c], p1[c], y, M, N, K, ws)
+
+    if not a.time:
+        for i in range(a.launches):
+            call(i)
+        torch.cuda.synchronize()
+        print(json.dumps({"launches": a.launches, "error_flags": qlinear_read_error(ws)}))
+        return
+    for i in range(2 * a.copies):
+        call(i)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for i in range(a.launches):
+            call(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 10
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * a.launches)
+    b = algorithmic_bytes(fmt, K, N, M)
+    print(json.dumps({"fmt": a.fmt, "K": K, "N": N, "M": M, "us": round(us, 3), "bytes": b,
+                      "GBs": round(b / us / 1e3, 1), "ctas": qlinear_plan(fmt, M, N, K).ctas,
+                      "error_flags": qlinear_read_error(ws)}))
+
+
+if __name__ == "__main__":
+    main()
