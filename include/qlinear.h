@@ -166,6 +166,21 @@ ql_status qlinear_w4a16_outlier(const uint16_t* x, const uint32_t* qweight,
                                 int group, void* workspace, size_t workspace_bytes,
                                 ql_stream_t stream);
 
+/* The W4A16 GEMV of qlinear_w4a16 for callers that cannot allocate device memory (e.g. a
+ * plug-in whose device memory belongs to a host application or a fixed pool, or code that
+ * must not call cudaMalloc/cudaFree because they synchronize or are not allowed where it
+ * runs).  No page describes this entry; it has no counterpart in the method.
+ * Same arguments as qlinear_w4a16 without the workspace: the split-K scratch is a fixed
+ * 4 MiB array inside the library (on every device, from library load to process exit).
+ * It allocates nothing and frees nothing.  Returns QL_ERR_WORKSPACE if a call would need
+ * more than that scratch.  The first call on a device looks up the scratch's device
+ * address (make it before any stream capture).  Every call on a device shares the
+ * scratch: calls whose device work overlaps in time race and must not be issued;
+ * each call clears the parts that must start at zero on `stream` before its launch. */
+ql_status qlinear_w4a16_noalloc(const uint16_t* x, const uint32_t* qweight,
+                                const uint16_t* scales, const uint16_t* zeros, uint16_t* y,
+                                int M, int N, int K, int group, ql_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * Debug entries (device pointers, asynchronous).  They decode the packed layout
  * with the same fragment-extraction code the GEMV kernels use.

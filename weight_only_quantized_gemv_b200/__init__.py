@@ -58,6 +58,7 @@ _SIGS = {
     "qlinear_debug_dequant": (_I, [_I, _P, _P, _P, _P, _I, _I, _P]),
     "qlinear_plan": (_I, [_I, _I, _I, _I, ctypes.POINTER(ql_plan)]),
     "qlinear_read_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint32), _P]),
+    "qlinear_w4a16_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -183,6 +184,13 @@ def qlinear_w2a16(x, qweight, scales, zeros, y, M, N, K, workspace, stream=None,
 
 def qlinear_w8a16(x, qweight, scales, zeros, y, M, N, K, workspace, stream=None, group=128):
     return _uniform("qlinear_w8a16", x, qweight, scales, zeros, y, M, N, K, workspace, stream, group)
+
+
+def qlinear_w4a16_noalloc(x, qweight, scales, zeros, y, M, N, K, stream=None, group=128):
+    """qlinear_w4a16 with the library's fixed device scratch instead of a workspace."""
+    _check(_lib.qlinear_w4a16_noalloc(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(y),
+                                      M, N, K, group, _stream(stream)), "qlinear_w4a16_noalloc")
+    return y
 
 
 def qlinear_lut4(x, codes, lut16, absmax, y, M, N, K, workspace, stream=None, block=64):

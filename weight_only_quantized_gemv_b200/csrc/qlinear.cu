@@ -387,3 +387,68 @@ extern "C" ql_status qlinear_read_error(void* workspace, uint32_t* flags, ql_str
   if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), st) != cudaSuccess) return QL_ERR_CUDA;
   return cudaStreamSynchronize(st) == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------
+// W4A16 GEMV without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at all: plug-ins and embedded runtimes
+// whose device memory is owned by a host application or a fixed pool they may not grow,
+// and code that must not call cudaMalloc/cudaFree because those calls synchronize the
+// device or are forbidden in its execution context.  For them this entry point keeps its
+// split-K scratch (error word, arrival counters, partial sums) in a fixed array compiled
+// into the library instead of a workspace argument.
+//
+// The array lives in every device's memory from the moment the library is loaded until
+// the process exits.  In host code its name only stands in for it; the device address is
+// looked up once per device with cudaGetSymbolAddress, with that device current, on the
+// first call made on that device (so that first call should come before any stream
+// capture).  All calls on a device share the array and it keeps the contents of the last
+// call: the error word and the counters are cleared on the call's stream before each
+// launch, and two calls whose device work overlaps (e.g. on two streams) race on it.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_noalloc_scratch on the current device (looked up once per device).
+cudaError_t noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" ql_status qlinear_w4a16_noalloc(const uint16_t* x, const uint32_t* qweight,
+                                           const uint16_t* scales, const uint16_t* zeros,
+                                           uint16_t* y, int M, int N, int K, int group,
+                                           ql_stream_t stream) {
+  if (group != kGroup) return QL_ERR_SHAPE;
+  if (!x || !qweight || !scales || !zeros || !y) return QL_ERR_NULL;
+  if (!shape_ok(M, N, K)) return QL_ERR_SHAPE;
+  Plan p;
+  if (make_plan(kW4, M, N, K, false, &p) != cudaSuccess) return QL_ERR_CUDA;
+  if (p.ws_bytes > kNoAllocScratchBytes) return QL_ERR_WORKSPACE;  // beyond the fixed scratch
+  void* scratch = nullptr;
+  if (noalloc_scratch(&scratch) != cudaSuccess) return QL_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // error word and arrival counters must start at zero (the partial sums need not)
+  if (cudaMemsetAsync(scratch, 0, p.partial_offset, st) != cudaSuccess) return QL_ERR_CUDA;
+  Call c{kW4, false, x, qweight, scales, zeros, nullptr, nullptr, nullptr, y, M, N, K,
+         scratch, kNoAllocScratchBytes, st};
+  return run(c);
+}
