@@ -214,6 +214,32 @@ __device__ __forceinline__ uint16_t lds16(uint32_t a) {
   return v;
 }
 
+// Split-K arrival: atomic add at GPU scope with acquire-release semantics, returns the old value.
+__device__ __forceinline__ uint32_t arrive_acq_rel(uint32_t* counter) {
+  uint32_t old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(counter) : "memory");
+  return old;
+}
+
+__device__ __forceinline__ float4 ld_relaxed_gpu(const float4* p) {
+  float4 v;
+  asm volatile("ld.relaxed.gpu.global.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
+// Programmatic dependent launch: let the next kernel in the stream start (it still waits
+// for this grid to complete before it reads anything this grid wrote) / wait until the
+// previous kernel in the stream has completed and its writes are visible.
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void consumer_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
@@ -527,16 +553,17 @@ struct Gemv {
       for (int e = 0; e < NACC; e += 4)
         *reinterpret_cast<float4*>(dst + (size_t)i * 32 * NACC + e) =
             make_float4(v[i][e], v[i][e + 1], v[i][e + 2], v[i][e + 3]);
-    __threadfence();
+    // the warp's stores, then one acquire-release arrival: it publishes them (release) and,
+    // for the last contributor, makes every other contributor's partial visible (acquire)
     __syncwarp();
     uint32_t prev = 0;
-    if (lane == 0) prev = atomicAdd(P.counters + (size_t)b * NC + warp, 1u);
+    if (lane == 0) prev = arrive_acq_rel(P.counters + (size_t)b * NC + warp);
     prev = __shfl_sync(0xffffffffu, prev, 0);
     const int ub = b * P.G;
     const int cf = cta_of_unit(ub, P.U, P.C);
     const int cl = cta_of_unit(ub + P.G - 1, P.U, P.C);
     if (prev + 1 != (uint32_t)(cl - cf + 1)) return;
-    __threadfence();
+    __syncwarp();
     float s[T][NACC];
 #pragma unroll
     for (int i = 0; i < T; ++i)
@@ -556,7 +583,7 @@ struct Gemv {
           for (int i = 0; i < T; ++i)
 #pragma unroll
             for (int e = 0; e < NACC; e += 4)
-              q[f][i][e / 4] = __ldcg(reinterpret_cast<const float4*>(src + (size_t)i * 32 * NACC + e));
+              q[f][i][e / 4] = ld_relaxed_gpu(reinterpret_cast<const float4*>(src + (size_t)i * 32 * NACC + e));
         }
       }
 #pragma unroll
@@ -578,24 +605,23 @@ struct Gemv {
     if (lane == 0) P.counters[(size_t)b * NC + warp] = 0u;  // ready for the next call
   }
 
-  // Producer: one lane streams the CTA's units through the ring.
+  // Producer: one lane streams the CTA's units through the ring.  The packed weights and
+  // parameters of the first S units are requested before griddepcontrol.wait (they are
+  // static, so this may overlap the tail of the kernel before us in the stream); x, which
+  // that kernel may have produced, only after it.
   __device__ static void produce(const GemvParams& P, uint8_t* smem, int u0, int n) {
     const uint32_t ring = smem_addr(smem);
     const uint32_t bars = ring + C_::kBarOff;
     const uint64_t pol = evict_first_policy();
-    int b = u0 / P.G, g = u0 - b * P.G;
-    for (int i = 0; i < n; ++i) {
+    auto weights = [&](int i, int b, int g) {
       const int s = i % S;
-      if (i >= S && !mbar_wait(bars + 8 * (S + s), ((i / S) - 1) & 1))
-        atomicOr(P.err, kErrEmptyTimeout);
       const int tb = tiles_in_block(b, P.ntiles);
       const long long ch = chunk_index(b, g, 0, P.G, P.ntiles);
       const uint32_t st = ring + s * C_::kStageBytes;
       const uint32_t full = bars + 8 * s;
       const uint32_t code_bytes = tb * C_::kChunkBytes;
       const uint32_t param_bytes = tb * C_::kParamChunk;
-      const uint32_t x_bytes = 256u * P.M;
-      mbar_arrive_expect_tx(full, code_bytes + (kLut ? 1 : 2) * param_bytes + x_bytes);
+      mbar_arrive_expect_tx(full, code_bytes + (kLut ? 1 : 2) * param_bytes + 256u * P.M);
       bulk_g2s(st, P.qw + ch * C_::kChunkBytes, code_bytes, full, pol);
       if constexpr (kLut) {
         bulk_g2s(st + C_::kCodeBytes, static_cast<const float*>(P.zp) + ch * 32, param_bytes, full,
@@ -605,9 +631,33 @@ struct Gemv {
         bulk_g2s(st + C_::kCodeBytes + 256, static_cast<const __half*>(P.zp) + ch * 16,
                  param_bytes, full, pol);
       }
+    };
+    auto activations = [&](int i, int g) {
+      const int s = i % S;
+      const uint32_t st = ring + s * C_::kStageBytes;
       const __half* xg = P.x + (size_t)g * kGroup;
       for (int m = 0; m < P.M; ++m)
-        bulk_g2s(st + C_::kXOff + m * C_::kXStride, xg + (size_t)m * P.K, 256u, full);
+        bulk_g2s(st + C_::kXOff + m * C_::kXStride, xg + (size_t)m * P.K, 256u, bars + 8 * s);
+    };
+    const int b0 = u0 / P.G, g0 = u0 - b0 * P.G;
+    int b = b0, g = g0;
+    const int pre = n < S ? n : S;
+    for (int i = 0; i < pre; ++i) {
+      weights(i, b, g);
+      if (++g == P.G) {
+        g = 0;
+        ++b;
+      }
+    }
+    grid_dependency_wait();
+    b = b0;
+    g = g0;
+    for (int i = 0; i < n; ++i) {
+      if (i >= S) {
+        if (!mbar_wait(bars + 8 * (S + i % S), ((i / S) - 1) & 1)) atomicOr(P.err, kErrEmptyTimeout);
+        weights(i, b, g);
+      }
+      activations(i, g);
       if (++g == P.G) {
         g = 0;
         ++b;
@@ -752,14 +802,14 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, OUTL>::kThreads, Cfg<FMT, MT, OUT
     build_lut_table(reinterpret_cast<uint32_t*>(smem + C_::kLutOff), P.sc, threadIdx.x,
                     C_::kThreads);
   }
-  // x rows M .. kXRows-1 of every stage are never copied: keep them zero
+  // x rows M .. kXRows-1 of every stage are never copied: keep them zero (16-byte stores,
+  // rows are 272 = 17 x 16 bytes)
   {
-    constexpr int kRowWords = C_::kXStride / 4;
-    const int zrows = C_::kXRows > P.M ? C_::kXRows - P.M : 0;
-    const int per_stage = zrows * kRowWords;
-    for (int e = threadIdx.x; e < C_::S * per_stage; e += C_::kThreads) {
-      const int st = e / per_stage, r = e - st * per_stage;
-      reinterpret_cast<uint32_t*>(smem + st * C_::kStageBytes + C_::kXOff + P.M * C_::kXStride)[r] = 0u;
+    const int chunks = (C_::kXRows - (P.M < C_::kXRows ? P.M : C_::kXRows)) * (C_::kXStride / 16);
+#pragma unroll
+    for (int st = 0; st < C_::S; ++st) {
+      uint4* z = reinterpret_cast<uint4*>(smem + st * C_::kStageBytes + C_::kXOff + P.M * C_::kXStride);
+      for (int e = threadIdx.x; e < chunks; e += C_::kThreads) z[e] = make_uint4(0, 0, 0, 0);
     }
   }
   if constexpr (OUTL) {
@@ -769,10 +819,12 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, OUTL>::kThreads, Cfg<FMT, MT, OUT
     for (int i = threadIdx.x; i <= n; i += C_::kThreads) toff[i] = __ldg(P.tile_off + u0 + i);
   }
   __syncthreads();
+  grid_dependents_launch();
   if (warp == C_::NC) {
     if (lane == 0) G_::produce(P, smem, u0, n);
     return;
   }
+  grid_dependency_wait();  // x, y and the workspace may belong to the kernel before us
   G_::consume(P, smem, u0, n, warp, lane);
 }
 

@@ -176,7 +176,19 @@ ql_status run(const Call& c) {
   P.C = p.C;
   P.mul_shr8 = 1u << 24;
   const KernelInfo k = select_kernel(c.fmt, p.MT, c.outl);
-  k.fn<<<p.C, k.threads, k.smem, c.stream>>>(P);
+  // Programmatic stream serialization: the kernel may start while the previous kernel in
+  // the stream drains; it requests only static weight bytes before griddepcontrol.wait.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.C);
+  cfg.blockDim = dim3((unsigned)k.threads);
+  cfg.dynamicSmemBytes = (size_t)k.smem;
+  cfg.stream = c.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k.fn, P) != cudaSuccess) return QL_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
