@@ -95,11 +95,23 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
   p->ntiles = N / kTileN;
   p->nblocks = (p->ntiles + kBlockTiles - 1) / kBlockTiles;
   p->U = (long long)p->nblocks * p->G;
-  long long C = (long long)sms * occ;
-  // QLINEAR_MAX_CTAS caps the persistent grid (A/B runs, tests of the split-K fix-up)
+  const long long slots = (long long)sms * occ;  // CTAs resident at once
+  long long C = slots;
+  // Small layers (latency-bound: at most 16 units per CTA) use a block-aligned split when it
+  // fills most of the GPU: k CTAs per 128-column block with k | G gives every CTA a
+  // whole-group slice of one block, so each block has exactly k partial sums and no CTA
+  // straddles two blocks.  Larger layers stream over all resident slots (stream-K).
+  for (long long k = p->G; k >= 1; --k) {
+    if (p->G % k == 0 && p->nblocks * k <= slots) {
+      const long long ca = p->nblocks * k;
+      if (ca * 100 >= slots * 55 && p->U <= 16 * ca) C = ca;
+      break;
+    }
+  }
+  // QLINEAR_MAX_CTAS forces the grid size (A/B runs, tests of the split-K fix-up)
   if (const char* cap = getenv("QLINEAR_MAX_CTAS")) {
     const long long v = atoll(cap);
-    if (v > 0 && v < C) C = v;
+    if (v > 0) C = v;
   }
   if (outl) {  // a CTA keeps the Tile-COO offsets of its units in shared memory
     const long long cmin = (p->U + qlk::kMaxUnitsPerCta - 1) / qlk::kMaxUnitsPerCta;
