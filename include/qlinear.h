@@ -171,7 +171,7 @@ ql_status qlinear_w4a16_outlier(const uint16_t* x, const uint32_t* qweight,
  * must not call cudaMalloc/cudaFree because they synchronize or are not allowed where it
  * runs).  No page describes this entry; it has no counterpart in the method.
  * Same arguments as qlinear_w4a16 without the workspace: the split-K scratch is a fixed
- * 4 MiB array inside the library (on every device, from library load to process exit).
+ * 8 MiB array inside the library (on every device, from library load to process exit).
  * It allocates nothing and frees nothing.  Returns QL_ERR_WORKSPACE if a call would need
  * more than that scratch.  The first call on a device looks up the scratch's device
  * address (make it before any stream capture).  Every call on a device shares the

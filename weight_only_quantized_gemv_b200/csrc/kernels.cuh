@@ -108,13 +108,19 @@ __host__ __device__ constexpr int align_to(int v, int a) { return (v + a - 1) / 
 template <int FMT, int MT, bool OUTL>
 struct Cfg {
   static constexpr int NC = 4;                       // consumer warps
+  // warps that share each unit: one for 4-bit codes at M <= 8 (the least work per unit),
+  // else a pair, warp h of which takes tiles 4h .. 4h+3
+  static constexpr int WPU = (MT == 1 && FMT == kW4) ? 1 : 2;
+  static constexpr int NP = NC / WPU;                // warp groups, each takes whole units
+  static constexpr int kTW = kBlockTiles / WPU;      // tiles of a unit per warp
   static constexpr int T = 2;                        // tiles per warp in the block epilogue
   static constexpr int kThreads = (NC + 1) * 32;     // + one producer warp
   static constexpr int KW = Fmt<FMT>::kWords;
   static constexpr int NACC = 4 * MT;
-  // stages: a multiple of NC, warp w uses the stages s = w (mod NC)
-  static constexpr int S = NC * (MT == 1 ? Fmt<FMT>::kStagesPerWarpM8 : 2);
-  static constexpr int kMinCtas = (MT == 1 && FMT != kW8 && FMT != kLUT4) ? 3 : 1;
+  // stages: warp group p uses the stages s = p (mod NP); one per warp at M <= 8 (two for
+  // 2-bit codes, whose stages are small), two per group at M > 8
+  static constexpr int S = NC * (MT == 1 ? Fmt<FMT>::kStagesPerWarpM8 : (WPU == 1 ? 2 : 1));
+  static constexpr int kMinCtas = (FMT == kLUT4) ? 1 : (MT == 1 && FMT != kW8) ? 3 : 2;
   static constexpr int kChunkBytes = 128 * KW;
   static constexpr int kCodeBytes = kBlockTiles * kChunkBytes;
   static constexpr int kParamChunk = (FMT == kLUT4) ? 128 : 32;   // per tile, per array
@@ -128,7 +134,7 @@ struct Cfg {
   static constexpr int kLutOff = align_to(kBarOff + 16 * S, 128);
   static constexpr int kLutBytes = (FMT == kLUT4) ? 256 * 32 * 4 : 0;
   static constexpr int kRedOff = kLutOff + kLutBytes;              // per-warp block sums
-  static constexpr int kRedBytes = NC * kBlockTiles * 32 * NACC * 4;
+  static constexpr int kRedBytes = NC * kTW * 32 * NACC * 4;    // each warp holds kTW tiles
   static constexpr int kYsmOff = kRedOff + kRedBytes;
   static constexpr int kYsmBytes = OUTL ? 16 * 128 * 4 : 0;
   static constexpr int kToffOff = kYsmOff + kYsmBytes;
@@ -328,6 +334,7 @@ template <int FMT, int MT, bool OUTL>
 struct Gemv {
   using C_ = Cfg<FMT, MT, OUTL>;
   static constexpr int NC = C_::NC, T = C_::T, KW = C_::KW, NACC = C_::NACC, S = C_::S;
+  static constexpr int WPU = C_::WPU, NP = C_::NP, kTW = C_::kTW;
   static constexpr bool kLut = (FMT == kLUT4);
   static constexpr int kBT = kBlockTiles;
 
@@ -376,9 +383,9 @@ struct Gemv {
   }
 
   // MMAs and group epilogue of four tiles: four independent accumulator chains per step.
-  __device__ static void compute_quad(const Quad& r, int j0, int lane, uint32_t lut, uint32_t k24,
+  __device__ static void compute_quad(const Quad& r, int lane, uint32_t lut, uint32_t k24,
                                       const uint4 (&xr)[4], const uint4 (&xr2)[4],
-                                      const float (&cx)[NACC], float (&acc)[kBT][NACC]) {
+                                      const float (&cx)[NACC], float (*acc)[NACC]) {
     const auto& w = r.w;
     if constexpr (kLut) {
 #pragma unroll
@@ -407,8 +414,7 @@ struct Gemv {
           const float a0 = blk ? r.am[i].z : r.am[i].x;
           const float a8 = blk ? r.am[i].w : r.am[i].y;
 #pragma unroll
-          for (int e = 0; e < NACC; ++e)
-            acc[j0 + i][e] = fmaf((e & 2) ? a8 : a0, c[i][e], acc[j0 + i][e]);
+          for (int e = 0; e < NACC; ++e) acc[i][e] = fmaf((e & 2) ? a8 : a0, c[i][e], acc[i][e]);
         }
       }
     } else {
@@ -458,7 +464,7 @@ struct Gemv {
           if constexpr (FMT == kW2) d = fmaf(co[i][e], 0.0625f, d);  // odd steps carry x16
           const float sc = (e & 2) ? s2.y : s2.x;
           const float zc = (e & 2) ? z2.y : z2.x;
-          acc[j0 + i][e] = fmaf(sc, fmaf(-zc, cx[e], d), acc[j0 + i][e]);
+          acc[i][e] = fmaf(sc, fmaf(-zc, cx[e], d), acc[i][e]);
         }
       }
     }
@@ -485,21 +491,22 @@ struct Gemv {
   // tiles 2w, 2w+1), rescale, add outliers, write y or join the split-K fix-up.
   __device__ static void finish_block(const GemvParams& P, uint8_t* smem, int b, bool whole,
                                       int first_block, int warp, int lane,
-                                      float (&acc)[kBT][NACC]) {
+                                      float (&acc)[kTW][NACC]) {
     const int tb = tiles_in_block(b, P.ntiles);
     float* red = reinterpret_cast<float*>(smem + C_::kRedOff);
     float* ysm = reinterpret_cast<float*>(smem + C_::kYsmOff);
     consumer_sync(NC * 32);  // all units of the run are done (and their outliers in ysm)
 #pragma unroll
-    for (int j = 0; j < kBT; ++j) {
+    for (int j = 0; j < kTW; ++j) {
 #pragma unroll
       for (int e = 0; e < NACC; e += 4)
-        *reinterpret_cast<float4*>(red + ((warp * kBT + j) * 32 + lane) * NACC + e) =
+        *reinterpret_cast<float4*>(red + ((warp * kTW + j) * 32 + lane) * NACC + e) =
             make_float4(acc[j][e], acc[j][e + 1], acc[j][e + 2], acc[j][e + 3]);
 #pragma unroll
       for (int e = 0; e < NACC; ++e) acc[j][e] = 0.f;
     }
     consumer_sync(NC * 32);
+    // tile jj sits, in each warp group p, with warp WPU p + jj / kTW in slot jj % kTW
     float v[T][NACC];
 #pragma unroll
     for (int i = 0; i < T; ++i) {
@@ -507,11 +514,12 @@ struct Gemv {
 #pragma unroll
       for (int e = 0; e < NACC; ++e) v[i][e] = 0.f;
 #pragma unroll
-      for (int w2 = 0; w2 < NC; ++w2)
+      for (int p2 = 0; p2 < NP; ++p2)
 #pragma unroll
         for (int e = 0; e < NACC; e += 4) {
+          const int w2 = WPU * p2 + jj / kTW;
           const float4 q =
-              *reinterpret_cast<const float4*>(red + ((w2 * kBT + jj) * 32 + lane) * NACC + e);
+              *reinterpret_cast<const float4*>(red + ((w2 * kTW + jj % kTW) * 32 + lane) * NACC + e);
           v[i][e] += q.x;
           v[i][e + 1] += q.y;
           v[i][e + 2] += q.z;
@@ -665,13 +673,17 @@ struct Gemv {
     }
   }
 
-  // One unit (block b, group g) of the CTA's range, all its tiles, by one warp.
+  // One unit (block b, group g) of the CTA's range: warp h of the group takes tiles
+  // kTW h .. kTW h + kTW - 1 (of a ragged block, a warp without tiles only releases the
+  // stage; tiles past the block's end in a warp's last quad read stale bytes whose sums are
+  // never written out).
   __device__ static void unit(const GemvParams& P, uint8_t* smem, int i, int b, int warp,
-                              int lane, float (&acc)[kBT][NACC], uint32_t (&orc)[3],
+                              int lane, float (&acc)[kTW][NACC], uint32_t (&orc)[3],
                               uint32_t (&oval)[3], int n) {
     const uint32_t ring = smem_addr(smem);
     const uint32_t bars = ring + C_::kBarOff;
     const uint32_t lut = ring + C_::kLutOff;
+    const int sub = warp % WPU;
     const int s = i % S;
     const int tb = tiles_in_block(b, P.ntiles);
     const uint32_t st = ring + s * C_::kStageBytes;
@@ -679,63 +691,79 @@ struct Gemv {
     uint4 xr[4], xr2[4];
     read_x(P, st, lane, xr, xr2);
     if constexpr (OUTL) {
-      // outliers of this unit with x from the stage, then prefetch the warp's next unit's
-      float* ysm = reinterpret_cast<float*>(smem + C_::kYsmOff);
-      const uint32_t* toff = reinterpret_cast<const uint32_t*>(smem + C_::kToffOff);
-      const uint32_t e0 = toff[i] + lane, e1 = toff[i + 1];
-      auto add_outlier = [&](uint32_t rc, uint32_t vb) {
-        const int row = rc & 0xFF, col = rc >> 8;
-        const float v = __half2float(__ushort_as_half((unsigned short)vb));
-        const uint32_t xa = st + C_::kXOff + 2 * row;
-        for (int m = 0; m < P.M; ++m) {
-          const float xv = __half2float(__ushort_as_half(lds16(xa + m * C_::kXStride)));
-          atomicAdd(ysm + m * 128 + col, v * xv);
-        }
-      };
+      if (sub == 0) {
+        // outliers of this unit with x from the stage, then prefetch the group's next unit's
+        float* ysm = reinterpret_cast<float*>(smem + C_::kYsmOff);
+        const uint32_t* toff = reinterpret_cast<const uint32_t*>(smem + C_::kToffOff);
+        const uint32_t e0 = toff[i] + lane, e1 = toff[i + 1];
+        auto add_outlier = [&](uint32_t rc, uint32_t vb) {
+          const int row = rc & 0xFF, col = rc >> 8;
+          const float v = __half2float(__ushort_as_half((unsigned short)vb));
+          const uint32_t xa = st + C_::kXOff + 2 * row;
+          for (int m = 0; m < P.M; ++m) {
+            const float xv = __half2float(__ushort_as_half(lds16(xa + m * C_::kXStride)));
+            atomicAdd(ysm + m * 128 + col, v * xv);
+          }
+        };
 #pragma unroll
-      for (int k = 0; k < 3; ++k)
-        if (e0 + 32 * k < e1) add_outlier(orc[k], oval[k]);
-      for (uint32_t e = e0 + 96; e < e1; e += 32)  // tiles with more than 96 outliers
-        add_outlier(__ldg(P.tile_rc + e), __ldg(P.tile_val + e));
-      prefetch_outliers(P, toff, i + NC, n, lane, orc, oval);
-    }
-    float cx[NACC];
-    if constexpr (kLut) {
-#pragma unroll
-      for (int e = 0; e < NACC; ++e) cx[e] = 0.f;
-    } else {  // sum of x over the group, in the row scales of the codes
-      const uint32_t ones[4] = {kOnesLo, Fmt<FMT>::kOnesHi, kOnesLo, Fmt<FMT>::kOnesHi};
-      hmma0(&cx[0], ones, xr[0].x, xr[0].y);
-      if constexpr (MT == 2) hmma0(&cx[4], ones, xr2[0].x, xr2[0].y);
-#pragma unroll
-      for (int s8 = 1; s8 < 8; ++s8) {
-        const int p = s8 >> 1, h = s8 & 1;
-        hmma(&cx[0], ones, h ? xr[p].z : xr[p].x, h ? xr[p].w : xr[p].y);
-        if constexpr (MT == 2) hmma(&cx[4], ones, h ? xr2[p].z : xr2[p].x, h ? xr2[p].w : xr2[p].y);
+        for (int k = 0; k < 3; ++k)
+          if (e0 + 32 * k < e1) add_outlier(orc[k], oval[k]);
+        for (uint32_t e = e0 + 96; e < e1; e += 32)  // tiles with more than 96 outliers
+          add_outlier(__ldg(P.tile_rc + e), __ldg(P.tile_val + e));
+        prefetch_outliers(P, toff, i + NP, n, lane, orc, oval);
       }
     }
+    const int t0 = kTW * sub;                      // first tile of this warp
+    const int nq = tb <= t0 ? 0 : (tb - t0 >= kTW ? kTW / kQ : (tb - t0 + kQ - 1) / kQ);
     const uint32_t empty = bars + 8 * (S + s);
-    // Tiles 0..3, then 4..7 (of a ragged block some of the second four read stale bytes
-    // whose sums are never written out).  With M <= 8 all eight tiles fit in registers:
-    // the stage is released before any math, so the ring stays in flight.
-    // Tiles 0..3, then 4..7 (of a ragged block some of the second four read stale bytes
-    // whose sums are never written out).  The stage is released once the second
-    // four are in registers, so its refill overlaps their math.
-    {
-      Quad q0;
-      load_quad(st, 0, lane, q0);
-      if (tb <= kQ) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty);  // the unit's last shared-memory reads are issued
+    float cx[NACC];
+    auto sum_x = [&]() {
+      if constexpr (kLut) {
+#pragma unroll
+        for (int e = 0; e < NACC; ++e) cx[e] = 0.f;
+      } else {  // sum of x over the group, in the row scales of the codes
+        const uint32_t ones[4] = {kOnesLo, Fmt<FMT>::kOnesHi, kOnesLo, Fmt<FMT>::kOnesHi};
+        hmma0(&cx[0], ones, xr[0].x, xr[0].y);
+        if constexpr (MT == 2) hmma0(&cx[4], ones, xr2[0].x, xr2[0].y);
+#pragma unroll
+        for (int s8 = 1; s8 < 8; ++s8) {
+          const int p = s8 >> 1, h = s8 & 1;
+          hmma(&cx[0], ones, h ? xr[p].z : xr[p].x, h ? xr[p].w : xr[p].y);
+          if constexpr (MT == 2)
+            hmma(&cx[4], ones, h ? xr2[p].z : xr2[p].x, h ? xr2[p].w : xr2[p].y);
+        }
       }
-      compute_quad(q0, 0, lane, lut, P.mul_shr8, xr, xr2, cx, acc);
-    }
-    if (tb > kQ) {
-      Quad q1;
-      load_quad(st, kQ, lane, q1);
+    };
+    if constexpr (kTW == kQ) {
+      // one quad: into registers, release the stage, then the math
+      Quad q;
+      if (nq) load_quad(st, t0, lane, q);
       __syncwarp();
-      if (lane == 0) mbar_arrive(empty);
-      compute_quad(q1, kQ, lane, lut, P.mul_shr8, xr, xr2, cx, acc);
+      if (lane == 0) mbar_arrive(empty);  // this warp's reads of stage s are issued
+      if (!nq) return;
+      sum_x();
+      compute_quad(q, lane, lut, P.mul_shr8, xr, xr2, cx, acc);
+    } else {
+      // two quads: the stage is released once the last one is in registers, so its refill
+      // overlaps that quad's math
+      static_assert(kTW == 2 * kQ, "one or two quads per warp");
+      sum_x();
+      {
+        Quad q0;
+        load_quad(st, t0, lane, q0);
+        if (nq <= 1) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(empty);
+        }
+        compute_quad(q0, lane, lut, P.mul_shr8, xr, xr2, cx, acc);
+      }
+      if (nq > 1) {
+        Quad q1;
+        load_quad(st, t0 + kQ, lane, q1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty);
+        compute_quad(q1, lane, lut, P.mul_shr8, xr, xr2, cx, acc + kQ);
+      }
     }
   }
 
@@ -752,26 +780,28 @@ struct Gemv {
     }
   }
 
-  // Consumer warp `warp` takes units i = warp, warp + NC, ... of the CTA's range (the
-  // stages i mod S are then private to it), all tiles of each.  At the end of every
-  // run of units of one block the warps meet and combine their sums.
+  // Warp group p = warp / WPU takes units i = p, p + NP, ... of the CTA's range (the stages
+  // i mod S are then private to it).  At the end of every run of units of one block the
+  // warps meet and combine their sums.
   __device__ static void consume(const GemvParams& P, uint8_t* smem, int u0, int n,
                                  int warp, int lane) {
     const int first_block = u0 / P.G;
-    float acc[kBT][NACC];
+    const int grp = warp / WPU;
+    float acc[kTW][NACC];
 #pragma unroll
-    for (int j = 0; j < kBT; ++j)
+    for (int j = 0; j < kTW; ++j)
 #pragma unroll
       for (int e = 0; e < NACC; ++e) acc[j][e] = 0.f;
     uint32_t orc[3] = {0, 0, 0}, oval[3] = {0, 0, 0};
     if constexpr (OUTL)
-      prefetch_outliers(P, reinterpret_cast<const uint32_t*>(smem + C_::kToffOff), warp, n, lane,
-                        orc, oval);
+      if (warp % WPU == 0)
+        prefetch_outliers(P, reinterpret_cast<const uint32_t*>(smem + C_::kToffOff), grp, n, lane,
+                          orc, oval);
     int b = first_block, g0 = u0 - first_block * P.G;
     for (int i0 = 0; i0 < n; ++b) {
       const int len = (n - i0) < (P.G - g0) ? (n - i0) : (P.G - g0);
       const int i1 = i0 + len;
-      for (int i = i0 + ((warp - i0 % NC) + NC) % NC; i < i1; i += NC)
+      for (int i = i0 + ((grp - i0 % NP) + NP) % NP; i < i1; i += NP)
         unit(P, smem, i, b, warp, lane, acc, orc, oval, n);
       finish_block(P, smem, b, g0 == 0 && len == P.G, first_block, warp, lane, acc);
       i0 = i1;
@@ -794,7 +824,7 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, OUTL>::kThreads, Cfg<FMT, MT, OUT
     const uint32_t bars = smem_addr(smem) + C_::kBarOff;
     for (int s = 0; s < C_::S; ++s) {
       mbar_init(bars + 8 * s, 1);            // full: the producer's expect_tx arrival
-      mbar_init(bars + 8 * (C_::S + s), 1);  // empty: the one consumer warp of the stage
+      mbar_init(bars + 8 * (C_::S + s), C_::WPU);  // empty: the warps of the group
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }

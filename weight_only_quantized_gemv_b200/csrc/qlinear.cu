@@ -431,7 +431,7 @@ extern "C" ql_status qlinear_read_error(void* workspace, uint32_t* flags, ql_str
 // launch, and two calls whose device work overlaps (e.g. on two streams) race on it.
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
