@@ -155,9 +155,10 @@ ql_status run(const Call& c) {
   if (!shape_ok(c.M, c.N, c.K)) return QL_ERR_SHAPE;
   if (c.outl && c.N % 128) return QL_ERR_SHAPE;
   if (!aligned(c.x, 16) || !aligned(c.qw, 32) || !aligned(c.y, 2)) return QL_ERR_ALIGN;
+  // parameters arrive by bulk copies (16-byte aligned sources); the LUT is read directly
   if (c.fmt == kLUT4) {
     if (!aligned(c.p0, 2) || !aligned(c.p1, 16)) return QL_ERR_ALIGN;
-  } else if (!aligned(c.p0, 4) || !aligned(c.p1, 4)) {
+  } else if (!aligned(c.p0, 16) || !aligned(c.p1, 16)) {
     return QL_ERR_ALIGN;
   }
   if (c.outl && (!aligned(c.toff, 4) || !aligned(c.trc, 2) || !aligned(c.tval, 2)))
