@@ -124,6 +124,8 @@ def test_hot_path_validates_before_any_device_work(ql):
     assert call(M=0) == 2 and call(M=17) == 2
     assert call(N=24) == 2 and call(K=100) == 2 and call(g=64) == 2
     assert call(x=a + 2) == 3 and call(q=a + 16) == 3 and call(s=a + 2) == 3
+    # scales and zeros are bulk-copied: 16-byte aligned sources only
+    assert call(s=a + 4) == 3 and call(z=a + 8) == 3
     assert call(fn=lib.qlinear_w2a16, K=192) == 2
     assert call(fn=lib.qlinear_w8a16, N=8) == 2
     # LUT4 wants block 64
