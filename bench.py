@@ -440,7 +440,9 @@ def run_gpu(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    # default: about a second of timed GPU work (enough clock samples), and a bounded
+    # number of oracle samples for the reference arm
+    ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--ref-cols", type=int, default=16)
@@ -449,6 +451,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
+    if args.steps is None:
+        args.steps = 2000 if args.impl == "reference" else 10000
+    if args.steps < 1:
+        raise SystemExit("--steps must be at least 1")
     if args.impl == "reference":
         run_reference(args)
     else:

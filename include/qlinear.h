@@ -205,6 +205,7 @@ typedef struct {
   int tiles_per_warp;
   long long units;  /* (128-column block, 128-element group) work units */
   int m_bucket;     /* 1: M <= 8, 2: M <= 16 */
+  int warps_per_unit; /* consumer warps that share one work unit (1, 2 or 4) */
 } ql_plan;
 
 ql_status qlinear_plan(int fmt, int M, int N, int K, ql_plan* plan);

@@ -147,6 +147,32 @@ def test_split_k_partitions(kind, cap):
             os.environ["QLINEAR_MAX_CTAS"] = old
 
 
+@pytest.mark.parametrize("wpu", ["1", "2", "4"])
+@pytest.mark.parametrize("cap", ["0", "7", "29"])
+@pytest.mark.parametrize("M", [1, 5, 8])
+def test_w4_warps_per_unit(wpu, cap, M):
+    """Every W4 M <= 8 variant (1, 2 or 4 warps per unit), whole-block and split-K grids,
+    on a ragged block."""
+    K, N = 1408, 416
+    env = {"QLINEAR_WPU": wpu, "QLINEAR_MAX_CTAS": cap}
+    old = {k: os.environ.get(k) for k in env}
+    os.environ.update(env)
+    try:
+        u = uniform_layer(610, K, N, 4)
+        lay = layers.from_uniform(u, DEV)
+        x, xd = _x(611 + M, M, K)
+        ref = oracle.gemv_uniform(x, u.qweight, u.scales, u.zeros, 4, 128)
+        assert ql.qlinear_plan(4, M, N, K).warps_per_unit == int(wpu)
+        for _ in range(2):
+            assert_parity(_np(lay.forward(xd)), ref, what=f"w4 wpu={wpu} cap={cap} M={M}")
+    finally:
+        for k, v in old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+
+
 # ---------------------------------------------------------------------------
 # special cases
 

@@ -38,7 +38,8 @@ _SZ = ctypes.c_size_t
 
 class ql_plan(ctypes.Structure):
     _fields_ = [("ctas", ctypes.c_int), ("warps", ctypes.c_int), ("tiles_per_warp", ctypes.c_int),
-                ("units", ctypes.c_longlong), ("m_bucket", ctypes.c_int)]
+                ("units", ctypes.c_longlong), ("m_bucket", ctypes.c_int),
+                ("warps_per_unit", ctypes.c_int)]
 
 
 _SIGS = {

@@ -104,15 +104,21 @@ constexpr float kTwo24 = 16777216.0f;
 
 __host__ __device__ constexpr int align_to(int v, int a) { return (v + a - 1) / a * a; }
 
-// Shared-memory layout of one kernel instance.
-template <int FMT, int MT, bool OUTL>
+// Warps that share each unit by default: one for 4-bit codes at M <= 8 (the least work per
+// unit), else a pair.  The host may pick more for layers too small to keep every warp busy.
+__host__ __device__ constexpr int default_wpu(int fmt, int mt) { return (mt == 1 && fmt == kW4) ? 1 : 2; }
+
+// Shared-memory layout of one kernel instance.  WPU warps share each unit, warp h of a group
+// taking tiles (8 / WPU) h .. (8 / WPU) (h + 1) - 1.
+template <int FMT, int MT, bool OUTL, int WPU_>
 struct Cfg {
   static constexpr int NC = 4;                       // consumer warps
-  // warps that share each unit: one for 4-bit codes at M <= 8 (the least work per unit),
-  // else a pair, warp h of which takes tiles 4h .. 4h+3
-  static constexpr int WPU = (MT == 1 && FMT == kW4) ? 1 : 2;
+  static constexpr int WPU = WPU_;
+  static_assert(WPU == 1 || WPU == 2 || WPU == 4, "1, 2 or 4 warps per unit");
   static constexpr int NP = NC / WPU;                // warp groups, each takes whole units
   static constexpr int kTW = kBlockTiles / WPU;      // tiles of a unit per warp
+  // tiles a warp holds in registers at once (independent accumulator chains)
+  static constexpr int kQ = kTW < 4 ? kTW : 4;
   static constexpr int T = 2;                        // tiles per warp in the block epilogue
   static constexpr int kThreads = (NC + 1) * 32;     // + one producer warp
   static constexpr int KW = Fmt<FMT>::kWords;
@@ -120,7 +126,7 @@ struct Cfg {
   // stages: warp group p uses the stages s = p (mod NP); one per warp at M <= 8 (two for
   // 2-bit codes, whose stages are small), two per group at M > 8
   static constexpr int S = NC * (MT == 1 ? Fmt<FMT>::kStagesPerWarpM8 : (WPU == 1 ? 2 : 1));
-  static constexpr int kMinCtas = (FMT == kLUT4) ? 1 : (MT == 1 && FMT != kW8) ? 3 : 2;
+  static constexpr int kMinCtas = (FMT == kLUT4) ? (MT == 1 ? 2 : 1) : (MT == 1 && FMT != kW8) ? 3 : 2;
   static constexpr int kChunkBytes = 128 * KW;
   static constexpr int kCodeBytes = kBlockTiles * kChunkBytes;
   static constexpr int kParamChunk = (FMT == kLUT4) ? 128 : 32;   // per tile, per array
@@ -330,9 +336,9 @@ __host__ __device__ __forceinline__ int cta_of_unit(int u, int U, int C) {
 
 // ---------------------------------------------------------------------------
 
-template <int FMT, int MT, bool OUTL>
+template <int FMT, int MT, bool OUTL, int WPU_>
 struct Gemv {
-  using C_ = Cfg<FMT, MT, OUTL>;
+  using C_ = Cfg<FMT, MT, OUTL, WPU_>;
   static constexpr int NC = C_::NC, T = C_::T, KW = C_::KW, NACC = C_::NACC, S = C_::S;
   static constexpr int WPU = C_::WPU, NP = C_::NP, kTW = C_::kTW;
   static constexpr bool kLut = (FMT == kLUT4);
@@ -350,8 +356,8 @@ struct Gemv {
     }
   }
 
-  // The stage bytes of four tiles (j0 .. j0 + 3) of one unit, in registers.
-  static constexpr int kQ = 4;
+  // The stage bytes of kQ tiles (j0 .. j0 + kQ - 1) of one unit, in registers.
+  static constexpr int kQ = C_::kQ;
   struct Quad {
     uint32_t w[kQ][KW];
     uint32_t p0[kQ], p1[kQ];  // scale / zero pairs (uniform)
@@ -382,7 +388,7 @@ struct Gemv {
     }
   }
 
-  // MMAs and group epilogue of four tiles: four independent accumulator chains per step.
+  // MMAs and group epilogue of kQ tiles: kQ independent accumulator chains per step.
   __device__ static void compute_quad(const Quad& r, int lane, uint32_t lut, uint32_t k24,
                                       const uint4 (&xr)[4], const uint4 (&xr2)[4],
                                       const float (&cx)[NACC], float (*acc)[NACC]) {
@@ -810,11 +816,12 @@ struct Gemv {
   }
 };
 
-template <int FMT, int MT, bool OUTL>
-__global__ void __launch_bounds__(Cfg<FMT, MT, OUTL>::kThreads, Cfg<FMT, MT, OUTL>::kMinCtas)
+template <int FMT, int MT, bool OUTL, int WPU>
+__global__ void __launch_bounds__(Cfg<FMT, MT, OUTL, WPU>::kThreads,
+                                  Cfg<FMT, MT, OUTL, WPU>::kMinCtas)
     qgemv_kernel(const GemvParams P) {
-  using G_ = Gemv<FMT, MT, OUTL>;
-  using C_ = Cfg<FMT, MT, OUTL>;
+  using G_ = Gemv<FMT, MT, OUTL, WPU>;
+  using C_ = Cfg<FMT, MT, OUTL, WPU>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int u0 = unit_begin(blockIdx.x, P.U, P.C);

@@ -24,7 +24,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 struct Plan {
   int C;            // CTAs
   long long U;      // units
-  int nblocks, ntiles, G, MT, NC, T, threads, smem;
+  int nblocks, ntiles, G, MT, WPU, NC, T, threads, smem;
   size_t counter_offset, partial_offset, ws_bytes;
 };
 
@@ -35,17 +35,22 @@ struct KernelInfo {
   int threads, smem, NC, T;
 };
 
-template <int FMT, int MT, bool OUTL>
+template <int FMT, int MT, bool OUTL, int WPU = qlk::default_wpu(FMT, MT)>
 KernelInfo kernel_info() {
-  using C = qlk::Cfg<FMT, MT, OUTL>;
-  return KernelInfo{qlk::qgemv_kernel<FMT, MT, OUTL>, C::kThreads, C::kSmemBytes, C::NC, C::T};
+  using C = qlk::Cfg<FMT, MT, OUTL, WPU>;
+  return KernelInfo{qlk::qgemv_kernel<FMT, MT, OUTL, WPU>, C::kThreads, C::kSmemBytes, C::NC, C::T};
 }
 
-KernelInfo select_kernel(int fmt, int MT, bool outl) {
+// wpu: warps per unit; W4 at M <= 8 has the one-warp default and 2- and 4-warp variants for
+// small layers, every other kernel its default only.
+KernelInfo select_kernel(int fmt, int MT, bool outl, int wpu) {
   if (outl) return MT == 1 ? kernel_info<kW4, 1, true>() : kernel_info<kW4, 2, true>();
   switch (fmt) {
     case kW2: return MT == 1 ? kernel_info<kW2, 1, false>() : kernel_info<kW2, 2, false>();
-    case kW4: return MT == 1 ? kernel_info<kW4, 1, false>() : kernel_info<kW4, 2, false>();
+    case kW4:
+      if (MT == 2) return kernel_info<kW4, 2, false>();
+      return wpu == 4 ? kernel_info<kW4, 1, false, 4>()
+                      : wpu == 2 ? kernel_info<kW4, 1, false, 2>() : kernel_info<kW4, 1, false>();
     case kW8: return MT == 1 ? kernel_info<kW8, 1, false>() : kernel_info<kW8, 2, false>();
     default: return MT == 1 ? kernel_info<kLUT4, 1, false>() : kernel_info<kLUT4, 2, false>();
   }
@@ -83,7 +88,8 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   p->MT = M <= 8 ? 1 : 2;
-  const KernelInfo k = select_kernel(fmt, p->MT, outl);
+  p->WPU = qlk::default_wpu(fmt, p->MT);
+  const KernelInfo k = select_kernel(fmt, p->MT, outl, p->WPU);
   int occ = 1;
   e = prepare_kernel(k, dev, &occ);
   if (e != cudaSuccess) return e;
@@ -121,6 +127,27 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
   // the kernel's stream-K index arithmetic is 32-bit
   if (p->U * C >= (1LL << 31)) return cudaErrorInvalidValue;
   p->C = (int)C;
+  // W4 at M <= 8: a CTA with few units shares each unit among more warps, which shortens the
+  // one unit a warp would otherwise work through alone (QLINEAR_WPU = 1, 2 or 4 overrides)
+  if (fmt == kW4 && p->MT == 1 && !outl) {
+    const long long per_cta = (p->U + C - 1) / C;
+    int wpu = per_cta <= 4 ? 4 : per_cta <= 24 ? 2 : 1;
+    if (const char* w = getenv("QLINEAR_WPU")) {
+      const int v = atoi(w);
+      if (v == 1 || v == 2 || v == 4) wpu = v;
+    }
+    if (wpu != p->WPU) {
+      const KernelInfo k2 = select_kernel(fmt, p->MT, outl, wpu);
+      int occ2 = 1;
+      e = prepare_kernel(k2, dev, &occ2);
+      if (e != cudaSuccess) return e;
+      if (occ2 >= occ) {  // never fewer resident CTAs than the grid was sized for
+        p->WPU = wpu;
+        p->threads = k2.threads;
+        p->smem = k2.smem;
+      }
+    }
+  }
   p->counter_offset = kErrBytes;
   p->partial_offset = align_up(p->counter_offset + (size_t)p->nblocks * p->NC * sizeof(uint32_t), 256);
   p->ws_bytes = p->partial_offset +
@@ -188,7 +215,7 @@ ql_status run(const Call& c) {
   P.U = (int)p.U;
   P.C = p.C;
   P.mul_shr8 = 1u << 24;
-  const KernelInfo k = select_kernel(c.fmt, p.MT, c.outl);
+  const KernelInfo k = select_kernel(c.fmt, p.MT, c.outl, p.WPU);
   // Programmatic stream serialization: the kernel may start while the previous kernel in
   // the stream drains; it requests only static weight bytes before griddepcontrol.wait.
   cudaLaunchConfig_t cfg = {};
@@ -344,6 +371,7 @@ extern "C" ql_status qlinear_plan(int fmt, int M, int N, int K, ql_plan* plan) {
   plan->tiles_per_warp = p.T;
   plan->units = p.U;
   plan->m_bucket = p.MT;
+  plan->warps_per_unit = p.WPU;
   return QL_OK;
 }
 
