@@ -158,7 +158,10 @@ ql_status qlinear_lut4(const uint16_t* x, const uint8_t* codes, const uint16_t* 
  * block-major order): tile_offsets uint32[T+1] (4-byte aligned), tile_rc uint8[nnz][2]
  * (2-byte aligned), tile_vals fp16[nnz] (2-byte aligned), T = (K/128) * (N/128).
  * Needs N % 128 == 0.  The dense code of every outlier position should
- * hold its group's zero code (then the dense part contributes nothing there). */
+ * hold its group's zero code (then the dense part contributes nothing there).
+ * The offsets must be non-decreasing with tile_offsets[T] = nnz (qlinear_pack_tilecoo
+ * checks this; the hot path reads them as given).  In-tile rows and columns are taken
+ * modulo 128, so a malformed pair gives a wrong sum, never an access outside the tile. */
 ql_status qlinear_w4a16_outlier(const uint16_t* x, const uint32_t* qweight,
                                 const uint16_t* scales, const uint16_t* zeros,
                                 const uint32_t* tile_offsets, const uint8_t* tile_rc,

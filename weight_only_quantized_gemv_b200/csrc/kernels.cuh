@@ -697,27 +697,30 @@ struct Gemv {
     uint4 xr[4], xr2[4];
     read_x(P, st, lane, xr, xr2);
     if constexpr (OUTL) {
-      if (sub == 0) {
-        // outliers of this unit with x from the stage, then prefetch the group's next unit's
-        float* ysm = reinterpret_cast<float*>(smem + C_::kYsmOff);
-        const uint32_t* toff = reinterpret_cast<const uint32_t*>(smem + C_::kToffOff);
-        const uint32_t e0 = toff[i] + lane, e1 = toff[i + 1];
-        auto add_outlier = [&](uint32_t rc, uint32_t vb) {
-          const int row = rc & 0xFF, col = rc >> 8;
-          const float v = __half2float(__ushort_as_half((unsigned short)vb));
-          const uint32_t xa = st + C_::kXOff + 2 * row;
-          for (int m = 0; m < P.M; ++m) {
-            const float xv = __half2float(__ushort_as_half(lds16(xa + m * C_::kXStride)));
-            atomicAdd(ysm + m * 128 + col, v * xv);
-          }
-        };
+      // outliers of this unit, split over the warps of the group, with x from the stage;
+      // then prefetch the group's next unit's
+      float* ysm = reinterpret_cast<float*>(smem + C_::kYsmOff);
+      const uint32_t* toff = reinterpret_cast<const uint32_t*>(smem + C_::kToffOff);
+      const uint32_t e0 = toff[i] + 32 * sub + lane, e1 = toff[i + 1];
+      auto add_outlier = [&](uint32_t rc, uint32_t vb) {
+        // in-tile position; an out-of-range pair wraps instead of leaving the tile
+        const int row = rc & 0x7F, col = (rc >> 8) & 0x7F;
+        const float v = __half2float(__ushort_as_half((unsigned short)vb));
+        const uint32_t xa = st + C_::kXOff + 2 * row;
+        float xv[C_::kXRows];  // all rows' loads in flight before the first atomic
 #pragma unroll
-        for (int k = 0; k < 3; ++k)
-          if (e0 + 32 * k < e1) add_outlier(orc[k], oval[k]);
-        for (uint32_t e = e0 + 96; e < e1; e += 32)  // tiles with more than 96 outliers
-          add_outlier(__ldg(P.tile_rc + e), __ldg(P.tile_val + e));
-        prefetch_outliers(P, toff, i + NP, n, lane, orc, oval);
-      }
+        for (int m = 0; m < C_::kXRows; ++m)
+          xv[m] = m < P.M ? __half2float(__ushort_as_half(lds16(xa + m * C_::kXStride))) : 0.f;
+#pragma unroll
+        for (int m = 0; m < C_::kXRows; ++m)
+          if (m < P.M) atomicAdd(ysm + m * 128 + col, v * xv[m]);
+      };
+#pragma unroll
+      for (int k = 0; k < kOutPre; ++k)
+        if (e0 + 32 * WPU * k < e1) add_outlier(orc[k], oval[k]);
+      for (uint32_t e = e0 + 32 * WPU * kOutPre; e < e1; e += 32 * WPU)  // dense tiles
+        add_outlier(__ldg(P.tile_rc + e), __ldg(P.tile_val + e));
+      prefetch_outliers(P, toff, i + NP, n, 32 * sub + lane, orc, oval);
     }
     const int t0 = kTW * sub;                      // first tile of this warp
     const int nq = tb <= t0 ? 0 : (tb - t0 >= kTW ? kTW / kQ : (tb - t0 + kQ - 1) / kQ);
@@ -773,12 +776,15 @@ struct Gemv {
     }
   }
 
+  // Entries of unit i a thread takes first (index `slot` of the WPU x 32 threads of the
+  // group, then every WPU x 32-th), held in registers one unit ahead.
+  static constexpr int kOutPre = 3 - (WPU > 1) - (WPU > 2);
   __device__ static void prefetch_outliers(const GemvParams& P, const uint32_t* toff, int i, int n,
-                                           int lane, uint32_t (&orc)[3], uint32_t (&oval)[3]) {
+                                           int slot, uint32_t (&orc)[3], uint32_t (&oval)[3]) {
     if (i >= n) return;
 #pragma unroll
-    for (int k = 0; k < 3; ++k) {
-      const uint32_t e = toff[i] + lane + 32 * k;
+    for (int k = 0; k < kOutPre; ++k) {
+      const uint32_t e = toff[i] + slot + 32 * WPU * k;
       if (e < toff[i + 1]) {
         orc[k] = __ldg(P.tile_rc + e);
         oval[k] = __ldg(P.tile_val + e);
@@ -799,10 +805,11 @@ struct Gemv {
 #pragma unroll
       for (int e = 0; e < NACC; ++e) acc[j][e] = 0.f;
     uint32_t orc[3] = {0, 0, 0}, oval[3] = {0, 0, 0};
-    if constexpr (OUTL)
-      if (warp % WPU == 0)
-        prefetch_outliers(P, reinterpret_cast<const uint32_t*>(smem + C_::kToffOff), grp, n, lane,
-                          orc, oval);
+    if constexpr (OUTL) {
+      consumer_sync(NC * 32);  // the Tile-COO offsets are in shared memory
+      prefetch_outliers(P, reinterpret_cast<const uint32_t*>(smem + C_::kToffOff), grp, n,
+                        32 * (warp % WPU) + lane, orc, oval);
+    }
     int b = first_block, g0 = u0 - first_block * P.G;
     for (int i0 = 0; i0 < n; ++b) {
       const int len = (n - i0) < (P.G - g0) ? (n - i0) : (P.G - g0);
@@ -852,14 +859,18 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, OUTL, WPU>::kThreads,
   if constexpr (OUTL) {
     float* ysm = reinterpret_cast<float*>(smem + C_::kYsmOff);
     for (int i = threadIdx.x; i < 16 * 128; i += C_::kThreads) ysm[i] = 0.f;
-    uint32_t* toff = reinterpret_cast<uint32_t*>(smem + C_::kToffOff);
-    for (int i = threadIdx.x; i <= n; i += C_::kThreads) toff[i] = __ldg(P.tile_off + u0 + i);
   }
   __syncthreads();
   grid_dependents_launch();
   if (warp == C_::NC) {
     if (lane == 0) G_::produce(P, smem, u0, n);
     return;
+  }
+  if constexpr (OUTL) {
+    // the range's Tile-COO offsets (static data, like the weights), fetched while the
+    // first stages fill; consume() meets on a barrier before reading them
+    uint32_t* toff = reinterpret_cast<uint32_t*>(smem + C_::kToffOff);
+    for (int i = threadIdx.x; i <= n; i += C_::NC * 32) toff[i] = __ldg(P.tile_off + u0 + i);
   }
   grid_dependency_wait();  // x, y and the workspace may belong to the kernel before us
   G_::consume(P, smem, u0, n, warp, lane);

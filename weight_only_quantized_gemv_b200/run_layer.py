@@ -1,13 +1,14 @@
 """Run one quantized-GEMV configuration repeatedly (for timing and profiler captures).
 
     python -m weight_only_quantized_gemv_b200.run_layer --fmt w4 --K 8192 --N 28672 --M 1 \
-        --launches 4 [--copies 3] [--time]
+        --launches 4 [--copies 3] [--time] [--outliers 0.005]
 
 The packed codes and parameters are random bytes of the right sizes (the kernel's
 speed does not depend on their values), allocated in `--copies` copies that the
-launches cycle through so that no launch finds its weights in L2.  With `--time` the
-launches are replayed from a CUDA graph and the mean device time per launch is
-printed as JSON.
+launches cycle through so that no launch finds its weights in L2.  With `--outliers F`
+(W4 only) every 128 x 128 tile also carries round(F * 16384) Tile-COO entries at random
+in-tile positions, and the outlier-aware entry point runs.  With `--time` the launches
+are replayed from a CUDA graph and the mean device time per launch is printed as JSON.
 """
 from __future__ import annotations
 
@@ -17,15 +18,21 @@ import json
 import torch
 
 from . import (FORMATS, QL_FMT_LUT4, qlinear_lut4, qlinear_plan, qlinear_read_error,
-               qlinear_w2a16, qlinear_w4a16, qlinear_w8a16, qlinear_workspace_bytes)
+               qlinear_w2a16, qlinear_w4a16, qlinear_w4a16_outlier, qlinear_w8a16,
+               qlinear_workspace_bytes)
 
 _UNIFORM = {2: qlinear_w2a16, 4: qlinear_w4a16, 8: qlinear_w8a16}
 
 
-def algorithmic_bytes(fmt: int, K: int, N: int, M: int) -> int:
+def algorithmic_bytes(fmt: int, K: int, N: int, M: int, nnz: int = 0) -> int:
+    """Bytes a launch must move at least: codes, parameters, x and y (and the Tile-COO
+    arrays: 2-byte (row, col) and 2-byte value per outlier, 4-byte offset per tile)."""
     if fmt == QL_FMT_LUT4:
         return K * N // 2 + (K // 64) * N * 4 + 32 + M * K * 2 + M * N * 2
-    return K * N * fmt // 8 + 2 * (K // 128) * N * 2 + M * K * 2 + M * N * 2
+    b = K * N * fmt // 8 + 2 * (K // 128) * N * 2 + M * K * 2 + M * N * 2
+    if nnz:
+        b += 4 * nnz + 4 * ((K // 128) * (N // 128) + 1)
+    return b
 
 
 def main() -> None:
@@ -37,8 +44,11 @@ def main() -> None:
     ap.add_argument("--launches", type=int, default=4)
     ap.add_argument("--copies", type=int, default=3)
     ap.add_argument("--time", action="store_true")
+    ap.add_argument("--outliers", type=float, default=0.0)
     a = ap.parse_args()
     fmt, K, N, M = FORMATS[a.fmt], a.K, a.N, a.M
+    if a.outliers and (a.fmt != "w4" or N % 128):
+        raise SystemExit("--outliers needs --fmt w4 and N % 128 == 0")
     dev = torch.device("cuda:0")
     torch.cuda.set_device(dev)
     bits = 4 if fmt == QL_FMT_LUT4 else fmt
@@ -57,9 +67,23 @@ def main() -> None:
     x = torch.randn(M, K, device=dev, generator=gen).half().view(torch.int16)
     y = torch.empty(M, N, device=dev, dtype=torch.int16)
     ws = torch.zeros(qlinear_workspace_bytes(fmt, M, N, K) // 4 + 64, dtype=torch.int32, device=dev)
+    nnz = 0
+    outl = a.outliers > 0  # the outlier-aware entry, even if the density rounds to no entries
+    if outl:
+        T = (K // 128) * (N // 128)
+        per = int(round(a.outliers * 128 * 128))
+        nnz = per * T
+        toff = (torch.arange(T + 1, device=dev, dtype=torch.int64) * per).to(torch.int32)
+        trc = [torch.randint(0, 128, (max(nnz, 1) * 2,), dtype=torch.uint8, device=dev, generator=gen)
+               for _ in range(a.copies)]  # in-tile (row, col) pairs
+        tval = [(torch.randn(max(nnz, 1), device=dev, generator=gen) * 0.2).half().view(torch.int16)
+                for _ in range(a.copies)]
+
     def call(i):  # on the current stream (the capture stream inside the graph below)
         c = i % a.copies
-        if fmt == QL_FMT_LUT4:
+        if outl:
+            qlinear_w4a16_outlier(x, q[c], p0[c], p1[c], toff, trc[c], tval[c], y, M, N, K, ws)
+        elif fmt == QL_FMT_LUT4:
             qlinear_lut4(x, q[c], p0[c], p1[c], y, M, N, K, ws)
         else:
             _UNIFORM[fmt](x, q[c], p0[c], p1[c], y, M, N, K, ws)
@@ -88,8 +112,8 @@ def main() -> None:
     e1.record()
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / (reps * a.launches)
-    b = algorithmic_bytes(fmt, K, N, M)
-    print(json.dumps({"fmt": a.fmt, "K": K, "N": N, "M": M, "us": round(us, 3), "bytes": b,
+    b = algorithmic_bytes(fmt, K, N, M, nnz) + (4 * ((K // 128) * (N // 128) + 1) if outl and not nnz else 0)
+    print(json.dumps({"fmt": a.fmt, "K": K, "N": N, "M": M, "nnz": nnz, "us": round(us, 3), "bytes": b,
                       "GBs": round(b / us / 1e3, 1), "ctas": qlinear_plan(fmt, M, N, K).ctas,
                       "error_flags": qlinear_read_error(ws)}))
 
