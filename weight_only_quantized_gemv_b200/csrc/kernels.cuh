@@ -109,9 +109,12 @@ __host__ __device__ constexpr int align_to(int v, int a) { return (v + a - 1) / 
 __host__ __device__ constexpr int default_wpu(int fmt, int mt) { return (mt == 1 && fmt == kW4) ? 1 : 2; }
 
 // Shared-memory layout of one kernel instance.  WPU warps share each unit, warp h of a group
-// taking tiles (8 / WPU) h .. (8 / WPU) (h + 1) - 1.
-template <int FMT, int MT, bool OUTL, int WPU_>
+// taking tiles (8 / WPU) h .. (8 / WPU) (h + 1) - 1.  M1: exactly one row of x (only the
+// accumulator entries of batch column 0 are kept).
+template <int FMT, int MT, bool OUTL, int WPU_, bool M1_ = false>
 struct Cfg {
+  static constexpr bool M1 = M1_;
+  static_assert(!M1 || MT == 1, "one row of x is the M <= 8 bucket");
   static constexpr int NC = 4;                       // consumer warps
   static constexpr int WPU = WPU_;
   static_assert(WPU == 1 || WPU == 2 || WPU == 4, "1, 2 or 4 warps per unit");
@@ -336,9 +339,9 @@ __host__ __device__ __forceinline__ int cta_of_unit(int u, int U, int C) {
 
 // ---------------------------------------------------------------------------
 
-template <int FMT, int MT, bool OUTL, int WPU_>
+template <int FMT, int MT, bool OUTL, int WPU_, bool M1_ = false>
 struct Gemv {
-  using C_ = Cfg<FMT, MT, OUTL, WPU_>;
+  using C_ = Cfg<FMT, MT, OUTL, WPU_, M1_>;
   static constexpr int NC = C_::NC, T = C_::T, KW = C_::KW, NACC = C_::NACC, S = C_::S;
   static constexpr int WPU = C_::WPU, NP = C_::NP, kTW = C_::kTW;
   static constexpr bool kLut = (FMT == kLUT4);
@@ -466,6 +469,7 @@ struct Gemv {
         const float2 z2 = __half22float2(*reinterpret_cast<const __half2*>(&r.p1[i]));
 #pragma unroll
         for (int e = 0; e < NACC; ++e) {
+          if (C_::M1 && (e & 1)) continue;  // batch column 1 of the fragment: no such row
           float d = c[i][e];
           if constexpr (FMT == kW2) d = fmaf(co[i][e], 0.0625f, d);  // odd steps carry x16
           const float sc = (e & 2) ? s2.y : s2.x;
@@ -823,12 +827,12 @@ struct Gemv {
   }
 };
 
-template <int FMT, int MT, bool OUTL, int WPU>
-__global__ void __launch_bounds__(Cfg<FMT, MT, OUTL, WPU>::kThreads,
-                                  Cfg<FMT, MT, OUTL, WPU>::kMinCtas)
+template <int FMT, int MT, bool OUTL, int WPU, bool M1 = false>
+__global__ void __launch_bounds__(Cfg<FMT, MT, OUTL, WPU, M1>::kThreads,
+                                  Cfg<FMT, MT, OUTL, WPU, M1>::kMinCtas)
     qgemv_kernel(const GemvParams P) {
-  using G_ = Gemv<FMT, MT, OUTL, WPU>;
-  using C_ = Cfg<FMT, MT, OUTL, WPU>;
+  using G_ = Gemv<FMT, MT, OUTL, WPU, M1>;
+  using C_ = Cfg<FMT, MT, OUTL, WPU, M1>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int u0 = unit_begin(blockIdx.x, P.U, P.C);

@@ -25,6 +25,7 @@ struct Plan {
   int C;            // CTAs
   long long U;      // units
   int nblocks, ntiles, G, MT, WPU, NC, T, threads, smem;
+  bool M1;          // W4 with one row of x: the kernel keeps only batch column 0
   size_t counter_offset, partial_offset, ws_bytes;
 };
 
@@ -35,22 +36,27 @@ struct KernelInfo {
   int threads, smem, NC, T;
 };
 
-template <int FMT, int MT, bool OUTL, int WPU = qlk::default_wpu(FMT, MT)>
+template <int FMT, int MT, bool OUTL, int WPU = qlk::default_wpu(FMT, MT), bool M1 = false>
 KernelInfo kernel_info() {
-  using C = qlk::Cfg<FMT, MT, OUTL, WPU>;
-  return KernelInfo{qlk::qgemv_kernel<FMT, MT, OUTL, WPU>, C::kThreads, C::kSmemBytes, C::NC, C::T};
+  using C = qlk::Cfg<FMT, MT, OUTL, WPU, M1>;
+  return KernelInfo{qlk::qgemv_kernel<FMT, MT, OUTL, WPU, M1>, C::kThreads, C::kSmemBytes, C::NC,
+                    C::T};
 }
 
 // wpu: warps per unit; W4 at M <= 8 has the one-warp default and 2- and 4-warp variants for
-// small layers, every other kernel its default only.
-KernelInfo select_kernel(int fmt, int MT, bool outl, int wpu) {
+// small layers, every other kernel its default only.  m1: W4 with exactly one row of x.
+template <int WPU>
+KernelInfo w4_m8_kernel(bool m1) {
+  return m1 ? kernel_info<kW4, 1, false, WPU, true>() : kernel_info<kW4, 1, false, WPU, false>();
+}
+
+KernelInfo select_kernel(int fmt, int MT, bool outl, int wpu, bool m1) {
   if (outl) return MT == 1 ? kernel_info<kW4, 1, true>() : kernel_info<kW4, 2, true>();
   switch (fmt) {
     case kW2: return MT == 1 ? kernel_info<kW2, 1, false>() : kernel_info<kW2, 2, false>();
     case kW4:
       if (MT == 2) return kernel_info<kW4, 2, false>();
-      return wpu == 4 ? kernel_info<kW4, 1, false, 4>()
-                      : wpu == 2 ? kernel_info<kW4, 1, false, 2>() : kernel_info<kW4, 1, false>();
+      return wpu == 4 ? w4_m8_kernel<4>(m1) : wpu == 2 ? w4_m8_kernel<2>(m1) : w4_m8_kernel<1>(m1);
     case kW8: return MT == 1 ? kernel_info<kW8, 1, false>() : kernel_info<kW8, 2, false>();
     default: return MT == 1 ? kernel_info<kLUT4, 1, false>() : kernel_info<kLUT4, 2, false>();
   }
@@ -89,7 +95,8 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
   if (e != cudaSuccess) return e;
   p->MT = M <= 8 ? 1 : 2;
   p->WPU = qlk::default_wpu(fmt, p->MT);
-  const KernelInfo k = select_kernel(fmt, p->MT, outl, p->WPU);
+  p->M1 = fmt == kW4 && M == 1 && !outl;
+  const KernelInfo k = select_kernel(fmt, p->MT, outl, p->WPU, p->M1);
   int occ = 1;
   e = prepare_kernel(k, dev, &occ);
   if (e != cudaSuccess) return e;
@@ -137,7 +144,7 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
       if (v == 1 || v == 2 || v == 4) wpu = v;
     }
     if (wpu != p->WPU) {
-      const KernelInfo k2 = select_kernel(fmt, p->MT, outl, wpu);
+      const KernelInfo k2 = select_kernel(fmt, p->MT, outl, wpu, p->M1);
       int occ2 = 1;
       e = prepare_kernel(k2, dev, &occ2);
       if (e != cudaSuccess) return e;
@@ -215,7 +222,7 @@ ql_status run(const Call& c) {
   P.U = (int)p.U;
   P.C = p.C;
   P.mul_shr8 = 1u << 24;
-  const KernelInfo k = select_kernel(c.fmt, p.MT, c.outl, p.WPU);
+  const KernelInfo k = select_kernel(c.fmt, p.MT, c.outl, p.WPU, p.M1);
   // Programmatic stream serialization: the kernel may start while the previous kernel in
   // the stream drains; it requests only static weight bytes before griddepcontrol.wait.
   cudaLaunchConfig_t cfg = {};
