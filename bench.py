@@ -156,16 +156,33 @@ def dist_setup(n_gpus):
     return rank, world, local
 
 
-def init_pg(local, world):
+def init_pg(local, world, backend="nccl"):
+    """Process group of the N replicas (none for one).  Only the timing barriers and the
+    max over ranks of the device times use it: the replicas share no data."""
     if world == 1:
         return None
     import datetime
 
     import torch
     import torch.distributed as dist
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                            device_id=torch.device("cuda", local))
+    kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return dist
+
+
+def max_over_ranks(value, dist, device):
+    """The slowest rank's time (every rank gets it); the value itself with one rank."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(bytes_per_step_per_rank, world, ms, steps):
+    """Whole-job throughput: the bytes all ranks moved over the slowest rank's time."""
+    return bytes_per_step_per_rank * world / (ms * 1e-3 / steps) / 1e9
 
 
 # ---------------------------------------------------------------------------
@@ -318,10 +335,7 @@ def run_gpu(args):
         dist.barrier()
     ms = start.elapsed_time(stop)
     err = max(ql.qlinear_read_error(lay.workspace) for lay in lays)
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, dev)
     del g10, g1
 
     # per-layer breakdown: 30 launches of one layer over three copies of its packed weights
@@ -373,10 +387,7 @@ def run_gpu(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
 
     if rank == 0:
         peak, peak_src = measured_peaks()
@@ -396,7 +407,7 @@ def run_gpu(args):
         clocks = clk.summary()
         out = {
             "metric": METRIC,
-            "value": step_bytes * world / (ms * 1e-3 / args.steps) / 1e9,
+            "value": job_gbs(step_bytes, world, ms, args.steps),
             "unit": "GB/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -421,7 +432,7 @@ def run_gpu(args):
                          "kernel": "qgemv_kernel<W4, M<=8> (one launch per layer)",
                          "timing": "CUDA events around the timed region (graph replays of whole steps); "
                                    "the per-layer table comes from a separate 30-launch pass per layer"},
-            "e2e": {"value": step_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+            "e2e": {"value": job_gbs(step_bytes, world, e2e_ms, 1), "unit": "GB/s",
                     "h2d_bytes_per_step": int(sum(x.numel() * 2 for x in xs)),
                     "d2h_bytes_per_step": int(sum(y.numel() * 2 for y in ys)),
                     "ms_per_step": e2e_ms},
