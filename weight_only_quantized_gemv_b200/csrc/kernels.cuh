@@ -143,7 +143,10 @@ struct Cfg {
   static constexpr int kLutOff = align_to(kBarOff + 16 * S, 128);
   static constexpr int kLutBytes = (FMT == kLUT4) ? 256 * 32 * 4 : 0;
   static constexpr int kRedOff = kLutOff + kLutBytes;              // per-warp block sums
-  static constexpr int kRedBytes = NC * kTW * 32 * NACC * 4;    // each warp holds kTW tiles
+  // each warp holds kTW tiles; sized for kTW = 8 in every variant, so that all variants of a
+  // format ask for the same shared memory (consecutive launches of different variants then
+  // share one L1 / shared-memory split and overlap)
+  static constexpr int kRedBytes = NC * kBlockTiles * 32 * NACC * 4;
   static constexpr int kYsmOff = kRedOff + kRedBytes;
   static constexpr int kYsmBytes = OUTL ? 16 * 128 * 4 : 0;
   static constexpr int kToffOff = kYsmOff + kYsmBytes;

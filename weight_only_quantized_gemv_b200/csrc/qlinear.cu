@@ -134,11 +134,13 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
   // the kernel's stream-K index arithmetic is 32-bit
   if (p->U * C >= (1LL << 31)) return cudaErrorInvalidValue;
   p->C = (int)C;
-  // W4 at M <= 8: a CTA with few units shares each unit among more warps, which shortens the
-  // one unit a warp would otherwise work through alone (QLINEAR_WPU = 1, 2 or 4 overrides)
+  // W4 at 2 <= M <= 8: a CTA with few units shares each unit among more warps, which
+  // shortens the one unit a warp would otherwise work through alone.  The M = 1 kernel
+  // (half the epilogue) is fastest with one warp per unit on every layer measured.
+  // QLINEAR_WPU = 1, 2 or 4 overrides.
   if (fmt == kW4 && p->MT == 1 && !outl) {
     const long long per_cta = (p->U + C - 1) / C;
-    int wpu = per_cta <= 4 ? 4 : per_cta <= 24 ? 2 : 1;
+    int wpu = p->M1 ? 1 : per_cta <= 4 ? 4 : per_cta <= 24 ? 2 : 1;
     if (const char* w = getenv("QLINEAR_WPU")) {
       const int v = atoi(w);
       if (v == 1 || v == 2 || v == 4) wpu = v;
