@@ -312,10 +312,15 @@ __device__ __forceinline__ void frag_uniform(const uint32_t* w, int s, uint32_t 
 
 // LUT4: byte j of word s holds the two codes of fragment register j; the replicated
 // table gives the fp16 pair (lut[lo], lut[hi]) from the lane's own bank.
-__device__ __forceinline__ void frag_lut(uint32_t v, uint32_t tbl, int lane, uint32_t (&a)[4]) {
+// tbl_lane = table base + 4 lane.  Entry (byte, lane) sits at byte * 128 + 4 lane: the byte
+// comes out with one byte permute (ALU) and the address with one multiply-add (FMA pipe).
+__device__ __forceinline__ void frag_lut(uint32_t v, uint32_t tbl_lane, uint32_t (&a)[4]) {
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
-    a[j] = lds32(tbl + (((((v >> (8 * j)) & 0xFFu) << 5) | (uint32_t)lane) << 2));
+  for (int j = 0; j < 4; ++j) {
+    uint32_t byte;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(byte) : "r"(v), "r"(0x4440u | (uint32_t)j));
+    a[j] = lds32(byte * 128u + tbl_lane);
+  }
 }
 
 __device__ __forceinline__ void build_lut_table(uint32_t* tbl, const __half* lut16, int tid,
@@ -410,7 +415,7 @@ struct Gemv {
 #pragma unroll
           for (int i = 0; i < kQ; ++i) {
             uint32_t a[4];
-            frag_lut(w[i][s], lut, lane, a);
+            frag_lut(w[i][s], lut + 4u * (uint32_t)lane, a);
             const uint32_t b2 = h ? xr2[p].z : xr2[p].x, b3 = h ? xr2[p].w : xr2[p].y;
             if (s == 4 * blk) {
               hmma0(&c[i][0], a, b0, b1);

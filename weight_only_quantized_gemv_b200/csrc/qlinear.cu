@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(128) debug_kernel(const uint8_t* packed, const
   for (int s = 0; s < 8; ++s) {
     uint32_t a[4];
     if constexpr (FMT == kLUT4) {
-      if (DEQ) qlk::frag_lut(wv[s], (uint32_t)__cvta_generic_to_shared(tbl), lane, a);
+      if (DEQ) qlk::frag_lut(wv[s], (uint32_t)__cvta_generic_to_shared(tbl) + 4u * (uint32_t)lane, a);
       else a[0] = a[1] = a[2] = a[3] = 0u;
     } else {
       qlk::frag_uniform<FMT>(wv, s, 1u << 24, a);
