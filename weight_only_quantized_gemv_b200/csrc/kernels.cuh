@@ -143,10 +143,11 @@ struct Cfg {
   static constexpr int kLutOff = align_to(kBarOff + 16 * S, 128);
   static constexpr int kLutBytes = (FMT == kLUT4) ? 256 * 32 * 4 : 0;
   static constexpr int kRedOff = kLutOff + kLutBytes;              // per-warp block sums
-  // each warp holds kTW tiles; sized for kTW = 8 in every variant, so that all variants of a
-  // format ask for the same shared memory (consecutive launches of different variants then
-  // share one L1 / shared-memory split and overlap)
-  static constexpr int kRedBytes = NC * kBlockTiles * 32 * NACC * 4;
+  // each warp holds kTW tiles.  The W4 M <= 8 variants (1, 2 or 4 warps per unit) all size
+  // it for kTW = 8, so that they ask for the same shared memory: consecutive launches of
+  // different variants then share one L1 / shared-memory split and overlap.
+  static constexpr int kRedBytes =
+      NC * ((FMT == kW4 && MT == 1) ? kBlockTiles : kTW) * 32 * NACC * 4;
   static constexpr int kYsmOff = kRedOff + kRedBytes;
   static constexpr int kYsmBytes = OUTL ? 16 * 128 * 4 : 0;
   static constexpr int kToffOff = kYsmOff + kYsmBytes;
