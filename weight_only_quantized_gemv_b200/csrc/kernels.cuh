@@ -129,7 +129,7 @@ struct Cfg {
   // stages: warp group p uses the stages s = p (mod NP); one per warp at M <= 8 (two for
   // 2-bit codes, whose stages are small), two per group at M > 8
   static constexpr int S = NC * (MT == 1 ? Fmt<FMT>::kStagesPerWarpM8 : (WPU == 1 ? 2 : 1));
-  static constexpr int kMinCtas = (FMT == kLUT4) ? (MT == 1 ? 2 : 1) : (MT == 1 && FMT != kW8) ? 3 : 2;
+  static constexpr int kMinCtas = (FMT == kLUT4) ? 2 : (MT == 1 && FMT != kW8) ? 3 : 2;
   static constexpr int kChunkBytes = 128 * KW;
   static constexpr int kCodeBytes = kBlockTiles * kChunkBytes;
   static constexpr int kParamChunk = (FMT == kLUT4) ? 128 : 32;   // per tile, per array
