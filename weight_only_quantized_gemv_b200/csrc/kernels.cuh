@@ -111,7 +111,7 @@ __host__ __device__ constexpr int default_wpu(int fmt, int mt) { return (mt == 1
 // Shared-memory layout of one kernel instance.  WPU warps share each unit, warp h of a group
 // taking tiles (8 / WPU) h .. (8 / WPU) (h + 1) - 1.  M1: exactly one row of x (only the
 // accumulator entries of batch column 0 are kept).
-template <int FMT, int MT, bool OUTL, int WPU_, bool M1_ = false>
+template <int FMT, int MT, bool OUTL, int WPU_, bool M1_ = false, int OCC_ = 0>
 struct Cfg {
   static constexpr bool M1 = M1_;
   static_assert(!M1 || MT == 1, "one row of x is the M <= 8 bucket");
@@ -129,7 +129,9 @@ struct Cfg {
   // stages: warp group p uses the stages s = p (mod NP); one per warp at M <= 8 (two for
   // 2-bit codes, whose stages are small), two per group at M > 8
   static constexpr int S = NC * (MT == 1 ? Fmt<FMT>::kStagesPerWarpM8 : (WPU == 1 ? 2 : 1));
-  static constexpr int kMinCtas = (FMT == kLUT4) ? 2 : (MT == 1 && FMT != kW8) ? 3 : 2;
+  // CTAs per SM the registers are sized for: OCC_, else the format's default (more CTAs,
+  // fewer registers per thread)
+  static constexpr int kMinCtas = OCC_ ? OCC_ : (FMT == kLUT4) ? 2 : (MT == 1 && FMT != kW8) ? 3 : 2;
   static constexpr int kChunkBytes = 128 * KW;
   static constexpr int kCodeBytes = kBlockTiles * kChunkBytes;
   static constexpr int kParamChunk = (FMT == kLUT4) ? 128 : 32;   // per tile, per array
@@ -348,9 +350,9 @@ __host__ __device__ __forceinline__ int cta_of_unit(int u, int U, int C) {
 
 // ---------------------------------------------------------------------------
 
-template <int FMT, int MT, bool OUTL, int WPU_, bool M1_ = false>
+template <int FMT, int MT, bool OUTL, int WPU_, bool M1_ = false, int OCC_ = 0>
 struct Gemv {
-  using C_ = Cfg<FMT, MT, OUTL, WPU_, M1_>;
+  using C_ = Cfg<FMT, MT, OUTL, WPU_, M1_, OCC_>;
   static constexpr int NC = C_::NC, T = C_::T, KW = C_::KW, NACC = C_::NACC, S = C_::S;
   static constexpr int WPU = C_::WPU, NP = C_::NP, kTW = C_::kTW;
   static constexpr bool kLut = (FMT == kLUT4);
@@ -836,12 +838,12 @@ struct Gemv {
   }
 };
 
-template <int FMT, int MT, bool OUTL, int WPU, bool M1 = false>
-__global__ void __launch_bounds__(Cfg<FMT, MT, OUTL, WPU, M1>::kThreads,
-                                  Cfg<FMT, MT, OUTL, WPU, M1>::kMinCtas)
+template <int FMT, int MT, bool OUTL, int WPU, bool M1 = false, int OCC = 0>
+__global__ void __launch_bounds__(Cfg<FMT, MT, OUTL, WPU, M1, OCC>::kThreads,
+                                  Cfg<FMT, MT, OUTL, WPU, M1, OCC>::kMinCtas)
     qgemv_kernel(const GemvParams P) {
-  using G_ = Gemv<FMT, MT, OUTL, WPU, M1>;
-  using C_ = Cfg<FMT, MT, OUTL, WPU, M1>;
+  using G_ = Gemv<FMT, MT, OUTL, WPU, M1, OCC>;
+  using C_ = Cfg<FMT, MT, OUTL, WPU, M1, OCC>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int u0 = unit_begin(blockIdx.x, P.U, P.C);

@@ -26,6 +26,7 @@ struct Plan {
   long long U;      // units
   int nblocks, ntiles, G, MT, WPU, NC, T, threads, smem;
   bool M1;          // W4 with one row of x: the kernel keeps only batch column 0
+  bool OCC2;        // ... with registers for two CTAs per SM (grids of at most 2 per SM)
   size_t counter_offset, partial_offset, ws_bytes;
 };
 
@@ -36,21 +37,25 @@ struct KernelInfo {
   int threads, smem, NC, T;
 };
 
-template <int FMT, int MT, bool OUTL, int WPU = qlk::default_wpu(FMT, MT), bool M1 = false>
+template <int FMT, int MT, bool OUTL, int WPU = qlk::default_wpu(FMT, MT), bool M1 = false,
+          int OCC = 0>
 KernelInfo kernel_info() {
-  using C = qlk::Cfg<FMT, MT, OUTL, WPU, M1>;
-  return KernelInfo{qlk::qgemv_kernel<FMT, MT, OUTL, WPU, M1>, C::kThreads, C::kSmemBytes, C::NC,
-                    C::T};
+  using C = qlk::Cfg<FMT, MT, OUTL, WPU, M1, OCC>;
+  return KernelInfo{qlk::qgemv_kernel<FMT, MT, OUTL, WPU, M1, OCC>, C::kThreads, C::kSmemBytes,
+                    C::NC, C::T};
 }
 
 // wpu: warps per unit; W4 at M <= 8 has the one-warp default and 2- and 4-warp variants for
 // small layers, every other kernel its default only.  m1: W4 with exactly one row of x.
+// occ2: the one-warp M = 1 kernel with registers for two CTAs per SM instead of three.
 template <int WPU>
 KernelInfo w4_m8_kernel(bool m1) {
   return m1 ? kernel_info<kW4, 1, false, WPU, true>() : kernel_info<kW4, 1, false, WPU, false>();
 }
 
-KernelInfo select_kernel(int fmt, int MT, bool outl, int wpu, bool m1) {
+KernelInfo select_kernel(int fmt, int MT, bool outl, int wpu, bool m1, bool occ2 = false) {
+  if (occ2 && fmt == kW4 && MT == 1 && !outl && wpu == 1 && m1)
+    return kernel_info<kW4, 1, false, 1, true, 2>();
   if (outl) return MT == 1 ? kernel_info<kW4, 1, true>() : kernel_info<kW4, 2, true>();
   switch (fmt) {
     case kW2: return MT == 1 ? kernel_info<kW2, 1, false>() : kernel_info<kW2, 2, false>();
@@ -96,6 +101,7 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
   p->MT = M <= 8 ? 1 : 2;
   p->WPU = qlk::default_wpu(fmt, p->MT);
   p->M1 = fmt == kW4 && M == 1 && !outl;
+  p->OCC2 = false;
   const KernelInfo k = select_kernel(fmt, p->MT, outl, p->WPU, p->M1);
   int occ = 1;
   e = prepare_kernel(k, dev, &occ);
@@ -119,6 +125,24 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
       const long long ca = p->nblocks * k;
       if (ca * 100 >= slots * 55 && p->U <= 16 * ca) C = ca;
       break;
+    }
+  }
+  // W4 at M = 1 has a variant with registers for two CTAs per SM (fewer spills).  On small
+  // layers a block-aligned grid of at most two CTAs per SM running it beats three:
+  //  - the largest k | G with nblocks * k <= 2 SMs keeps every CTA's share of its block
+  //    equal;
+  //  - if that leaves over a fifth of the two-per-SM slots idle, take the most CTAs per
+  //    block that fit instead: C = nblocks * k is still block-aligned, because CTA c covers
+  //    units [c G / k, (c + 1) G / k) of block c / k.
+  bool small_m1 = false;
+  if (p->M1) {
+    const long long c2 = 2LL * sms, kmax = c2 / p->nblocks;
+    if (kmax >= 1 && p->U <= 16 * p->nblocks * kmax) {
+      long long kd = kmax;
+      while (p->G % kd) --kd;
+      const long long k = (p->nblocks * kd * 5 >= c2 * 4) ? kd : kmax;
+      C = p->nblocks * k;
+      small_m1 = true;
     }
   }
   // QLINEAR_MAX_CTAS forces the grid size (A/B runs, tests of the split-K fix-up)
@@ -154,6 +178,19 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
         p->WPU = wpu;
         p->threads = k2.threads;
         p->smem = k2.smem;
+      }
+    }
+    // A grid of at most two CTAs per SM leaves the third slot empty: then the M = 1 kernel
+    // with more registers per thread (fewer spills) is faster.
+    if (p->M1 && p->WPU == 1 && (small_m1 || C <= 2LL * sms)) {
+      const KernelInfo k3 = select_kernel(fmt, p->MT, outl, 1, true, true);
+      int occ3 = 1;
+      e = prepare_kernel(k3, dev, &occ3);
+      if (e != cudaSuccess) return e;
+      if ((long long)occ3 * sms >= C) {
+        p->OCC2 = true;
+        p->threads = k3.threads;
+        p->smem = k3.smem;
       }
     }
   }
@@ -224,7 +261,7 @@ ql_status run(const Call& c) {
   P.U = (int)p.U;
   P.C = p.C;
   P.mul_shr8 = 1u << 24;
-  const KernelInfo k = select_kernel(c.fmt, p.MT, c.outl, p.WPU, p.M1);
+  const KernelInfo k = select_kernel(c.fmt, p.MT, c.outl, p.WPU, p.M1, p.OCC2);
   // Programmatic stream serialization: the kernel may start while the previous kernel in
   // the stream drains; it requests only static weight bytes before griddepcontrol.wait.
   cudaLaunchConfig_t cfg = {};
