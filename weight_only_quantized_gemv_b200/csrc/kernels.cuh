@@ -41,6 +41,7 @@
 //    workspace error word and carries on, so a lost copy can corrupt results but
 //    never hang the GPU.
 #pragma once
+#include <cuda.h>  // CUtensorMap
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -110,7 +111,8 @@ __host__ __device__ constexpr int default_wpu(int fmt, int mt) { return (mt == 1
 
 // Shared-memory layout of one kernel instance.  WPU warps share each unit, warp h of a group
 // taking tiles (8 / WPU) h .. (8 / WPU) (h + 1) - 1.  M1: exactly one row of x (only the
-// accumulator entries of batch column 0 are kept).
+// accumulator entries of batch column 0 are kept; x arrives by a 1-D bulk copy).  Every
+// other instance serves M >= 2 and copies x as one 2-D tile per unit through a tensor map.
 template <int FMT, int MT, bool OUTL, int WPU_, bool M1_ = false, int OCC_ = 0>
 struct Cfg {
   static constexpr bool M1 = M1_;
@@ -136,7 +138,9 @@ struct Cfg {
   static constexpr int kCodeBytes = kBlockTiles * kChunkBytes;
   static constexpr int kParamChunk = (FMT == kLUT4) ? 128 : 32;   // per tile, per array
   static constexpr int kParamBytes = (FMT == kLUT4) ? 8 * 128 : 2 * 8 * 32;
-  static constexpr int kXStride = 272;                             // 256 + 16 pad (banks)
+  // x rows in a stage: the 2-D tile copy (M >= 2) writes them densely; the single-row
+  // kernel keeps 16 bytes of padding, which spreads the fragment loads over the banks
+  static constexpr int kXStride = M1 ? 272 : 256;
   static constexpr int kXRows = 8 * MT;
   static constexpr int kXOff = kCodeBytes + kParamBytes;
   static constexpr int kStageBytes = align_to(kXOff + kXRows * kXStride, 128);
@@ -434,7 +438,8 @@ struct Gemv {
           const float a0 = blk ? r.am[i].z : r.am[i].x;
           const float a8 = blk ? r.am[i].w : r.am[i].y;
 #pragma unroll
-          for (int e = 0; e < NACC; ++e) acc[i][e] = fmaf((e & 2) ? a8 : a0, c[i][e], acc[i][e]);
+          for (int e = 0; e < NACC; ++e)
+            if (!C_::M1 || !(e & 1)) acc[i][e] = fmaf((e & 2) ? a8 : a0, c[i][e], acc[i][e]);
         }
       }
     } else {
@@ -638,7 +643,9 @@ struct Gemv {
   // parameters of the first S units are requested before griddepcontrol.wait (they are
   // static, so this may overlap the tail of the kernel before us in the stream); x, which
   // that kernel may have produced, only after it.
-  __device__ static void produce(const GemvParams& P, uint8_t* smem, int u0, int n) {
+  // xmap: the tensor map of x (kernels for M >= 2), in the kernel's parameter space
+  __device__ static void produce(const GemvParams& P, const CUtensorMap* xmap, uint8_t* smem,
+                                 int u0, int n) {
     const uint32_t ring = smem_addr(smem);
     const uint32_t bars = ring + C_::kBarOff;
     const uint64_t pol = evict_first_policy();
@@ -661,12 +668,24 @@ struct Gemv {
                  param_bytes, full, pol);
       }
     };
+    // the group's M rows of x: one row by a plain bulk copy; M >= 2 rows by one 2-D tensor
+    // copy of the box (k = 128 g .. 128 g + 127, every row), 128 g elements being a
+    // 256-byte aligned start
     auto activations = [&](int i, int g) {
       const int s = i % S;
       const uint32_t st = ring + s * C_::kStageBytes;
-      const __half* xg = P.x + (size_t)g * kGroup;
-      for (int m = 0; m < P.M; ++m)
-        bulk_g2s(st + C_::kXOff + m * C_::kXStride, xg + (size_t)m * P.K, 256u, bars + 8 * s);
+      if constexpr (C_::M1) {
+        const __half* xg = P.x + (size_t)g * kGroup;
+        for (int m = 0; m < P.M; ++m)
+          bulk_g2s(st + C_::kXOff + m * C_::kXStride, xg + (size_t)m * P.K, 256u, bars + 8 * s);
+      } else {
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3}], [%4];"
+            :: "r"(st + C_::kXOff), "l"(reinterpret_cast<uint64_t>(xmap)), "r"(g * kGroup),
+               "r"(0), "r"(bars + 8 * s)
+            : "memory");
+      }
     };
     const int b0 = u0 / P.G, g0 = u0 - b0 * P.G;
     int b = b0, g = g0;
@@ -838,10 +857,21 @@ struct Gemv {
   }
 };
 
-template <int FMT, int MT, bool OUTL, int WPU, bool M1 = false, int OCC = 0>
+// Second kernel parameter: the tensor map of x for the kernels of M >= 2, an unused word for
+// the single-row ones.  (Kept out of GemvParams: a 128-byte grid-constant parameter block
+// costs the single-row kernels about 3%.)
+struct NoXMap {
+  int unused;
+};
+template <bool XT> struct XMapParam { using type = NoXMap; };
+template <> struct XMapParam<true> { using type = CUtensorMap; };
+
+template <int FMT, int MT, bool OUTL, int WPU, bool M1, int OCC>
 __global__ void __launch_bounds__(Cfg<FMT, MT, OUTL, WPU, M1, OCC>::kThreads,
                                   Cfg<FMT, MT, OUTL, WPU, M1, OCC>::kMinCtas)
-    qgemv_kernel(const GemvParams P) {
+    qgemv_kernel(const GemvParams P, const __grid_constant__ typename XMapParam<!M1>::type xm) {
+  const CUtensorMap* xmap = nullptr;
+  if constexpr (!M1) xmap = &xm;
   using G_ = Gemv<FMT, MT, OUTL, WPU, M1, OCC>;
   using C_ = Cfg<FMT, MT, OUTL, WPU, M1, OCC>;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -862,7 +892,7 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, OUTL, WPU, M1, OCC>::kThreads,
                     C_::kThreads);
   }
   // x rows M .. kXRows-1 of every stage are never copied: keep them zero (16-byte stores,
-  // rows are 272 = 17 x 16 bytes)
+  // rows are 256 bytes)
   {
     const int chunks = (C_::kXRows - (P.M < C_::kXRows ? P.M : C_::kXRows)) * (C_::kXStride / 16);
 #pragma unroll
@@ -878,7 +908,7 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, OUTL, WPU, M1, OCC>::kThreads,
   __syncthreads();
   grid_dependents_launch();
   if (warp == C_::NC) {
-    if (lane == 0) G_::produce(P, smem, u0, n);
+    if (lane == 0) G_::produce(P, xmap, smem, u0, n);
     return;
   }
   if constexpr (OUTL) {
@@ -890,5 +920,6 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, OUTL, WPU, M1, OCC>::kThreads,
   grid_dependency_wait();  // x, y and the workspace may belong to the kernel before us
   G_::consume(P, smem, u0, n, warp, lane);
 }
+
 
 }  // namespace qlk

@@ -1,5 +1,7 @@
 // C ABI of the quantized GEMV library: argument checks, launch planning, kernel
 // instances and the debug decode kernels.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -30,19 +32,25 @@ struct Plan {
   size_t counter_offset, partial_offset, ws_bytes;
 };
 
-using KernelPtr = void (*)(qlk::GemvParams);
-
 struct KernelInfo {
-  KernelPtr fn;
+  const void* fn;  // qgemv_kernel<...>: its second parameter a tensor map of x if xt
   int threads, smem, NC, T;
+  bool xt;
 };
 
 template <int FMT, int MT, bool OUTL, int WPU = qlk::default_wpu(FMT, MT), bool M1 = false,
           int OCC = 0>
 KernelInfo kernel_info() {
   using C = qlk::Cfg<FMT, MT, OUTL, WPU, M1, OCC>;
-  return KernelInfo{qlk::qgemv_kernel<FMT, MT, OUTL, WPU, M1, OCC>, C::kThreads, C::kSmemBytes,
-                    C::NC, C::T};
+  return KernelInfo{reinterpret_cast<const void*>(qlk::qgemv_kernel<FMT, MT, OUTL, WPU, M1, OCC>),
+                    C::kThreads, C::kSmemBytes, C::NC, C::T, !M1};
+}
+
+// The M <= 8 kernel of a format: its single-row variant for M = 1, else the one for M >= 2.
+template <int FMT, bool OUTL>
+KernelInfo m8_kernel(bool m1) {
+  return m1 ? kernel_info<FMT, 1, OUTL, qlk::default_wpu(FMT, 1), true>()
+            : kernel_info<FMT, 1, OUTL>();
 }
 
 // wpu: warps per unit; W4 at M <= 8 has the one-warp default and 2- and 4-warp variants for
@@ -56,14 +64,14 @@ KernelInfo w4_m8_kernel(bool m1) {
 KernelInfo select_kernel(int fmt, int MT, bool outl, int wpu, bool m1, bool occ2 = false) {
   if (occ2 && fmt == kW4 && MT == 1 && !outl && wpu == 1 && m1)
     return kernel_info<kW4, 1, false, 1, true, 2>();
-  if (outl) return MT == 1 ? kernel_info<kW4, 1, true>() : kernel_info<kW4, 2, true>();
+  if (outl) return MT == 1 ? m8_kernel<kW4, true>(m1) : kernel_info<kW4, 2, true>();
   switch (fmt) {
-    case kW2: return MT == 1 ? kernel_info<kW2, 1, false>() : kernel_info<kW2, 2, false>();
+    case kW2: return MT == 1 ? m8_kernel<kW2, false>(m1) : kernel_info<kW2, 2, false>();
     case kW4:
       if (MT == 2) return kernel_info<kW4, 2, false>();
       return wpu == 4 ? w4_m8_kernel<4>(m1) : wpu == 2 ? w4_m8_kernel<2>(m1) : w4_m8_kernel<1>(m1);
-    case kW8: return MT == 1 ? kernel_info<kW8, 1, false>() : kernel_info<kW8, 2, false>();
-    default: return MT == 1 ? kernel_info<kLUT4, 1, false>() : kernel_info<kLUT4, 2, false>();
+    case kW8: return MT == 1 ? m8_kernel<kW8, false>(m1) : kernel_info<kW8, 2, false>();
+    default: return MT == 1 ? m8_kernel<kLUT4, false>(m1) : kernel_info<kLUT4, 2, false>();
   }
 }
 
@@ -100,7 +108,7 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
   if (e != cudaSuccess) return e;
   p->MT = M <= 8 ? 1 : 2;
   p->WPU = qlk::default_wpu(fmt, p->MT);
-  p->M1 = fmt == kW4 && M == 1 && !outl;
+  p->M1 = M == 1;
   p->OCC2 = false;
   const KernelInfo k = select_kernel(fmt, p->MT, outl, p->WPU, p->M1);
   int occ = 1;
@@ -135,7 +143,7 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
   //    block that fit instead: C = nblocks * k is still block-aligned, because CTA c covers
   //    units [c G / k, (c + 1) G / k) of block c / k.
   bool small_m1 = false;
-  if (p->M1) {
+  if (p->M1 && fmt == kW4 && !outl) {
     const long long c2 = 2LL * sms, kmax = c2 / p->nblocks;
     if (kmax >= 1 && p->U <= 16 * p->nblocks * kmax) {
       long long kd = kmax;
@@ -199,6 +207,37 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
   p->ws_bytes = p->partial_offset +
                 (size_t)2 * p->C * p->NC * p->T * 32 * 4 * p->MT * sizeof(float);
   return cudaSuccess;
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (no link
+// against libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// x [M][K] fp16 as a 2-D tensor (K innermost), box 128 x M: one copy brings a group's
+// 128 elements of every row.  x is 16-byte aligned and the row stride 2K bytes a multiple of
+// 256, as the copy requires.
+bool encode_x_map(CUtensorMap* map, const void* x, int M, int K) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kGroup, (cuuint32_t)M};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(x), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool shape_ok(int M, int N, int K) {
@@ -274,7 +313,16 @@ ql_status run(const Call& c) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, k.fn, P) != cudaSuccess) return QL_ERR_CUDA;
+  if (k.xt) {
+    CUtensorMap xmap;
+    if (!encode_x_map(&xmap, c.x, c.M, c.K)) return QL_ERR_CUDA;
+    void* args[2] = {&P, &xmap};
+    if (cudaLaunchKernelExC(&cfg, k.fn, args) != cudaSuccess) return QL_ERR_CUDA;
+  } else {
+    qlk::NoXMap none{0};
+    void* args[2] = {&P, &none};
+    if (cudaLaunchKernelExC(&cfg, k.fn, args) != cudaSuccess) return QL_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
