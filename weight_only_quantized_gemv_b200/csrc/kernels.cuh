@@ -603,8 +603,11 @@ struct Gemv {
     for (int i = 0; i < T; ++i)
 #pragma unroll
       for (int e = 0; e < NACC; ++e) s[i][e] = 0.f;
-    // contributors in CTA order; loads of up to kF slots are in flight at once
-    constexpr int kF = 4;
+    // contributors in CTA order; loads of up to kF slots are in flight at once.  Kernels
+    // sized for three CTAs per SM (128 registers) load one at a time: the registers of a
+    // deeper batch, though only live here, cost the main loop more spills than the
+    // shallower fix-up costs (measured on the W4 layers of the step).
+    constexpr int kF = C_::kMinCtas >= 3 ? 1 : 4;
     for (int c0 = cf; c0 <= cl; c0 += kF) {
       float4 q[kF][T][NACC / 4];
 #pragma unroll
