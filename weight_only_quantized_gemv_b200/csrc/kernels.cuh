@@ -133,6 +133,7 @@ struct Cfg {
   static constexpr int S = NC * (MT == 1 ? Fmt<FMT>::kStagesPerWarpM8 : (WPU == 1 ? 2 : 1));
   // CTAs per SM the registers are sized for: OCC_, else the format's default (more CTAs,
   // fewer registers per thread)
+  static constexpr int kOcc = OCC_;
   static constexpr int kMinCtas = OCC_ ? OCC_ : (FMT == kLUT4) ? 2 : (MT == 1 && FMT != kW8) ? 3 : 2;
   static constexpr int kChunkBytes = 128 * KW;
   static constexpr int kCodeBytes = kBlockTiles * kChunkBytes;
@@ -603,11 +604,11 @@ struct Gemv {
     for (int i = 0; i < T; ++i)
 #pragma unroll
       for (int e = 0; e < NACC; ++e) s[i][e] = 0.f;
-    // contributors in CTA order; loads of up to kF slots are in flight at once.  Kernels
-    // sized for three CTAs per SM (128 registers) load one at a time: the registers of a
-    // deeper batch, though only live here, cost the main loop more spills than the
-    // shallower fix-up costs (measured on the W4 layers of the step).
-    constexpr int kF = C_::kMinCtas >= 3 ? 1 : 4;
+    // contributors in CTA order; loads of up to kF slots are in flight at once.  One at a
+    // time, except in the small-layer variant: the registers of a deeper batch, though only
+    // live here, cost the main loop more spills than the shallower fix-up costs, and only
+    // small layers (many contributors per block, little work) feel the fix-up's latency.
+    constexpr int kF = C_::kOcc == 2 ? 4 : 1;
     for (int c0 = cf; c0 <= cl; c0 += kF) {
       float4 q[kF][T][NACC / 4];
 #pragma unroll
