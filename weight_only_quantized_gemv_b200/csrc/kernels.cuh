@@ -123,7 +123,7 @@ struct Cfg {
   static constexpr int NP = NC / WPU;                // warp groups, each takes whole units
   static constexpr int kTW = kBlockTiles / WPU;      // tiles of a unit per warp
   // tiles a warp holds in registers at once (independent accumulator chains)
-  static constexpr int kQ = kTW < 4 ? kTW : 4;
+  static constexpr int kQ = kTW < 4 ? kTW : (MT == 2 || FMT == kW8) ? 2 : 4;
   static constexpr int T = 2;                        // tiles per warp in the block epilogue
   static constexpr int kThreads = (NC + 1) * 32;     // + one producer warp
   static constexpr int KW = Fmt<FMT>::kWords;
