@@ -71,7 +71,6 @@ struct GemvParams {
   int M, N, K, G, nblocks, ntiles;
   int U;                      // nblocks * G
   int C;                      // CTAs
-  uint32_t mul_shr8;          // 2^24: v >> 8 as mul.hi on the FMA pipe (set by the host)
 };
 
 template <int FMT> struct Fmt;
@@ -291,18 +290,18 @@ __device__ __forceinline__ void hmma0(float* c, const uint32_t (&a)[4], uint32_t
 // A fragment (a0a1, a2a3, a4a5, a6a7) of step s from a lane's words.  For the uniform
 // formats each half holds code << shift, the shift fixed per register (layout.h):
 // W4 rows gi+8 carry x16, W2 rows gi+8 carry x4 and odd steps x16.
-__device__ __forceinline__ uint32_t shr8(uint32_t v, uint32_t) { return v >> 8; }
+__device__ __forceinline__ uint32_t shr8(uint32_t v) { return v >> 8; }
 
 template <int FMT>
-__device__ __forceinline__ void frag_uniform(const uint32_t* w, int s, uint32_t k24, uint32_t (&a)[4]) {
+__device__ __forceinline__ void frag_uniform(const uint32_t* w, int s, uint32_t (&a)[4]) {
   if constexpr (FMT == kW4) {
-    const uint32_t v = w[s], h = shr8(v, k24);
+    const uint32_t v = w[s], h = shr8(v);
     a[0] = v & 0x000F000Fu;  // row gi,   dk 0 | dk 1
     a[1] = v & 0x00F000F0u;  // row gi+8, dk 0 | dk 1
     a[2] = h & 0x000F000Fu;  // row gi,   dk 2 | dk 3
     a[3] = h & 0x00F000F0u;  // row gi+8, dk 2 | dk 3
   } else if constexpr (FMT == kW2) {
-    const uint32_t v = w[s >> 1], h = shr8(v, k24);
+    const uint32_t v = w[s >> 1], h = shr8(v);
     const uint32_t m0 = (s & 1) ? 0x00300030u : 0x00030003u;
     const uint32_t m1 = (s & 1) ? 0x00C000C0u : 0x000C000Cu;
     a[0] = v & m0;
@@ -313,8 +312,8 @@ __device__ __forceinline__ void frag_uniform(const uint32_t* w, int s, uint32_t 
     const uint32_t v0 = w[2 * s], v1 = w[2 * s + 1];
     a[0] = v0 & 0x00FF00FFu;
     a[1] = v1 & 0x00FF00FFu;
-    a[2] = shr8(v0, k24) & 0x00FF00FFu;
-    a[3] = shr8(v1, k24) & 0x00FF00FFu;
+    a[2] = shr8(v0) & 0x00FF00FFu;
+    a[3] = shr8(v1) & 0x00FF00FFu;
   }
 }
 
@@ -408,7 +407,7 @@ struct Gemv {
   }
 
   // MMAs and group epilogue of kQ tiles: kQ independent accumulator chains per step.
-  __device__ static void compute_quad(const Quad& r, int lane, uint32_t lut, uint32_t k24,
+  __device__ static void compute_quad(const Quad& r, int lane, uint32_t lut,
                                       const uint4 (&xr)[4], const uint4 (&xr2)[4],
                                       const float (&cx)[NACC], float (*acc)[NACC]) {
     const auto& w = r.w;
@@ -458,7 +457,7 @@ struct Gemv {
 #pragma unroll
         for (int i = 0; i < kQ; ++i) {
           uint32_t a[4];
-          frag_uniform<FMT>(w[i], s, k24, a);
+          frag_uniform<FMT>(w[i], s, a);
           if constexpr (FMT == kW2) {
             if (h == 1) {  // odd steps accumulate separately (their codes carry x16)
               if (s == 1) {
@@ -789,7 +788,7 @@ struct Gemv {
       if (lane == 0) mbar_arrive(empty);  // this warp's reads of stage s are issued
       if (!nq) return;
       sum_x();
-      compute_quad(q, lane, lut, P.mul_shr8, xr, xr2, cx, acc);
+      compute_quad(q, lane, lut, xr, xr2, cx, acc);
     } else {
       // two quads: the stage is released once the last one is in registers, so its refill
       // overlaps that quad's math
@@ -802,14 +801,14 @@ struct Gemv {
           __syncwarp();
           if (lane == 0) mbar_arrive(empty);
         }
-        compute_quad(q0, lane, lut, P.mul_shr8, xr, xr2, cx, acc);
+        compute_quad(q0, lane, lut, xr, xr2, cx, acc);
       }
       if (nq > 1) {
         Quad q1;
         load_quad(st, t0 + kQ, lane, q1);
         __syncwarp();
         if (lane == 0) mbar_arrive(empty);
-        compute_quad(q1, lane, lut, P.mul_shr8, xr, xr2, cx, acc + kQ);
+        compute_quad(q1, lane, lut, xr, xr2, cx, acc + kQ);
       }
     }
   }

@@ -299,7 +299,6 @@ ql_status run(const Call& c) {
   P.ntiles = p.ntiles;
   P.U = (int)p.U;
   P.C = p.C;
-  P.mul_shr8 = 1u << 24;
   const KernelInfo k = select_kernel(c.fmt, p.MT, c.outl, p.WPU, p.M1, p.OCC2);
   // Programmatic stream serialization: the kernel may start while the previous kernel in
   // the stream drains; it requests only static weight bytes before griddepcontrol.wait.
@@ -375,7 +374,7 @@ __global__ void __launch_bounds__(128) debug_kernel(const uint8_t* packed, const
       if (DEQ) qlk::frag_lut(wv[s], (uint32_t)__cvta_generic_to_shared(tbl) + 4u * (uint32_t)lane, a);
       else a[0] = a[1] = a[2] = a[3] = 0u;
     } else {
-      qlk::frag_uniform<FMT>(wv, s, 1u << 24, a);
+      qlk::frag_uniform<FMT>(wv, s, a);
     }
 #pragma unroll
     for (int r = 0; r < 4; ++r)
