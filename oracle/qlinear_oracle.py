@@ -25,7 +25,12 @@ Sources followed (page, section):
   Kernels" page, abstract and method section (NF4 codes turned back into
   values through a 16-entry table);
 * dense + sparse outlier decomposition ``y = x dequant(W_dense) + x W_out``:
-  FlashQuant page, English abstract.
+  FlashQuant page, English abstract;
+* stand-alone dequantization for prefill (fp16 weights written back to global
+  memory, then an ordinary fp16 matmul): "Fast NF4 Dequantization Kernels"
+  page, method section (technical framework: load codes, dequantize, write
+  FP16 back for the following computation); QFactory page, assumption stress
+  test and limitation 1 (prefill and large batches are compute-bound).
 
 Parity status: every function here is pinned by tests that do not re-state
 its formula (bounds against the unquantized weights, hand-derived golden
@@ -205,6 +210,36 @@ def gemv_outlier(x: np.ndarray, qweight: np.ndarray, scales: np.ndarray, zeros: 
     dense = gemv_uniform(x, qweight, scales, zeros, bits, group, cols)
     sparse = x.astype(np.float64) @ tilecoo_to_dense(offsets, rc, vals, K, N, cols)
     return dense + sparse
+
+
+# ---------------------------------------------------------------------------
+# stand-alone dequantization to fp16 + dense matmul (prefill, M >> 16)
+#
+# The fp16 weights are returned transposed, ``[N, K]`` (one row per output
+# column, the layout of a linear layer's weight matrix).  Readings taken:
+# a uniform weight is the exact ``s (q - z)`` rounded once to fp16 (round to
+# nearest even); a LUT4 weight is the fp32 product ``lut[q] * absmax`` rounded
+# to fp16, i.e. the fp32 dequantized value of the NF4 page's method (the
+# codebook value times the block absmax in fp32) stored as FP16.
+
+
+def dequant_uniform_fp16_nk(qweight: np.ndarray, scales: np.ndarray, zeros: np.ndarray,
+                            bits: int, group: int) -> np.ndarray:
+    """fp16 ``[N, K]``: ``fp16(s[k // g, n] * (q[k, n] - z[k // g, n]))`` transposed."""
+    w = dequant_uniform(unpack_uniform(qweight, bits), scales, zeros, group)
+    return np.ascontiguousarray(w.T).astype(np.float16)
+
+
+def dequant_lut4_fp16_nk(qbytes: np.ndarray, lut: np.ndarray, absmax: np.ndarray,
+                         block: int) -> np.ndarray:
+    """fp16 ``[N, K]``: ``fp16(fp32(lut[q[k, n]] * absmax[k // block, n]))`` transposed."""
+    w32 = dequant_lut4_fp32(unpack_lut4(qbytes), lut, absmax, block)
+    return np.ascontiguousarray(w32.T).astype(np.float16)
+
+
+def prefill_matmul(x: np.ndarray, w16_nk: np.ndarray) -> np.ndarray:
+    """``y[M, N] = x[M, K] @ W[N, K]^T`` in fp64 on the fp16 weights."""
+    return x.astype(np.float64) @ w16_nk.astype(np.float64).T
 
 
 # ---------------------------------------------------------------------------
