@@ -63,7 +63,8 @@ typedef enum {
   QL_ERR_ALIGN = 3,       /* a pointer is not aligned as documented */
   QL_ERR_UNSUPPORTED = 4, /* unknown format */
   QL_ERR_WORKSPACE = 5,   /* workspace missing or smaller than qlinear_workspace_bytes() */
-  QL_ERR_CUDA = 6         /* a CUDA runtime call or kernel launch failed */
+  QL_ERR_CUDA = 6,        /* a CUDA runtime call, kernel launch or cuBLAS call failed */
+  QL_ERR_LIBRARY = 7      /* cuBLAS (prefill GEMM) could not be opened or its handle created */
 } ql_status;
 
 typedef enum { QL_FMT_W2 = 2, QL_FMT_W4 = 4, QL_FMT_W8 = 8, QL_FMT_LUT4 = 16 } ql_format;
@@ -183,6 +184,41 @@ ql_status qlinear_w4a16_outlier(const uint16_t* x, const uint32_t* qweight,
 ql_status qlinear_w4a16_noalloc(const uint16_t* x, const uint32_t* qweight,
                                 const uint16_t* scales, const uint16_t* zeros, uint16_t* y,
                                 int M, int N, int K, int group, ql_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Prefill (M >> 16): stand-alone dequantization to fp16, then one dense GEMM.
+ * Source: "Fast NF4 Dequantization Kernels for Large Language Model Inference" page,
+ * method section (technical framework: load the codes, dequantize, write FP16 back to
+ * global memory for the following matmul; the 16-entry table lives in 64 bytes of
+ * shared memory); QFactory page, assumption stress test and limitation 1 (prefill and
+ * large batches are compute-bound, where the fused GEMV stops paying).
+ * ------------------------------------------------------------------------- */
+
+/* Dequantize packed weights into a dense fp16 matrix w[N][K] (row n = output column n,
+ * row stride K: the weight layout of a linear layer).  Device pointers, asynchronous on
+ * `stream`.
+ *   packed : packed codes (qlinear_pack), 16-byte aligned
+ *   p0, p1 : W2/W4/W8: packed scales and zeros (fp16, 4-byte aligned; zeros are integers
+ *            with |z| <= 1024);  LUT4: p0 = the fp16 lut[16] (2-byte aligned), p1 = the
+ *            packed fp32 absmax (16-byte aligned)
+ *   w      : fp16 [N][K], caller-allocated, 16-byte aligned, fully overwritten
+ * Values: W2/W4/W8 give fp16(s * (q - z)), the exact product rounded once to nearest even
+ * (overflow gives +-inf); LUT4 gives fp16(fp32(lut[q]) * absmax), the fp32 product rounded
+ * to fp32 and then to fp16.  N % 16 == 0, K % 128 == 0, N, K > 0 (QL_ERR_SHAPE otherwise). */
+ql_status qlinear_dequant_fp16(int fmt, const void* packed, const void* p0, const void* p1,
+                               uint16_t* w, int N, int K, ql_stream_t stream);
+
+/* y[M][N] = x[M][K] . w_fp16[N][K]^T for any M >= 1: qlinear_dequant_fp16 into the caller's
+ * w_fp16 (N * K * 2 bytes, 16-byte aligned, overwritten), then one cuBLAS GEMM on `stream`
+ * (fp16 operands and output, fp32 accumulation).  x and y are fp16 row-major device arrays
+ * (2-byte aligned; 16-byte alignment is faster).  cuBLAS is opened at run time
+ * (libcublas.so.12); the first call on a thread and device creates a cuBLAS handle, which
+ * allocates cuBLAS's own device memory and is kept for the life of the process: make that
+ * first call outside stream capture.  Returns QL_ERR_LIBRARY when cuBLAS cannot be opened
+ * or the handle cannot be created, QL_ERR_CUDA when the GEMM fails. */
+ql_status qlinear_prefill(int fmt, const uint16_t* x, const void* packed, const void* p0,
+                          const void* p1, uint16_t* w_fp16, uint16_t* y, int M, int N, int K,
+                          ql_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Debug entries (device pointers, asynchronous).  They decode the packed layout

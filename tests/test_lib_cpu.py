@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(ql):
 
 
 def test_status_strings(ql):
-    for s in range(7):
+    for s in range(8):
         assert ql._lib.ql_status_str(s)
     assert b"unknown" in ql._lib.ql_status_str(99)
 
@@ -142,3 +142,25 @@ def test_graft_entry_build_is_idempotent():
     import __graft_entry__ as ge
     ge.build()
     ge.build()
+
+
+def test_prefill_entries_validate_before_any_device_work(ql):
+    lib = ql._lib
+    a = 1 << 20
+    dq = lib.qlinear_dequant_fp16
+    assert dq(3, a, a, a, a, 128, 128, None) == 4
+    assert dq(4, None, a, a, a, 128, 128, None) == 1 and dq(4, a, a, a, None, 128, 128, None) == 1
+    assert dq(4, a, a, a, a, 24, 128, None) == 2 and dq(4, a, a, a, a, 128, 100, None) == 2
+    assert dq(4, a, a, a, a, 0, 128, None) == 2
+    assert dq(4, a + 8, a, a, a, 128, 128, None) == 3 and dq(4, a, a, a, a + 8, 128, 128, None) == 3
+    assert dq(4, a, a + 2, a, a, 128, 128, None) == 3 and dq(8, a, a, a + 2, a, 128, 128, None) == 3
+    assert dq(16, a, a, a + 4, a, 128, 128, None) == 3 and dq(16, a, a + 1, a, a, 128, 128, None) == 3
+    pf = lib.qlinear_prefill
+    assert pf(5, a, a, a, a, a, a, 64, 128, 128, None) == 4
+    assert pf(4, None, a, a, a, a, a, 64, 128, 128, None) == 1
+    assert pf(4, a, a, a, a, a, None, 64, 128, 128, None) == 1
+    assert pf(4, a, a, a, a, None, a, 64, 128, 128, None) == 1
+    assert pf(4, a, a, a, a, a, a, 0, 128, 128, None) == 2
+    assert pf(4, a, a, a, a, a, a, 64, 120, 128, None) == 2
+    assert pf(4, a + 1, a, a, a, a, a, 64, 128, 128, None) == 3
+    assert pf(4, a, a, a, a, a + 2, a, 64, 128, 128, None) == 3

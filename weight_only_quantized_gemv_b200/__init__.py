@@ -29,7 +29,8 @@ _lib = ctypes.CDLL(LIBRARY_PATH)
 QL_FMT_W2, QL_FMT_W4, QL_FMT_W8, QL_FMT_LUT4 = 2, 4, 8, 16
 FORMATS = {"w2": QL_FMT_W2, "w4": QL_FMT_W4, "w8": QL_FMT_W8, "lut4": QL_FMT_LUT4}
 STATUS = {0: "QL_OK", 1: "QL_ERR_NULL", 2: "QL_ERR_SHAPE", 3: "QL_ERR_ALIGN",
-          4: "QL_ERR_UNSUPPORTED", 5: "QL_ERR_WORKSPACE", 6: "QL_ERR_CUDA"}
+          4: "QL_ERR_UNSUPPORTED", 5: "QL_ERR_WORKSPACE", 6: "QL_ERR_CUDA",
+          7: "QL_ERR_LIBRARY"}
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -60,6 +61,8 @@ _SIGS = {
     "qlinear_plan": (_I, [_I, _I, _I, _I, ctypes.POINTER(ql_plan)]),
     "qlinear_read_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint32), _P]),
     "qlinear_w4a16_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "qlinear_dequant_fp16": (_I, [_I, _P, _P, _P, _P, _I, _I, _P]),
+    "qlinear_prefill": (_I, [_I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -223,3 +226,17 @@ def qlinear_debug_dequant(fmt, packed, p0, p1, w, N, K, stream=None):
     _check(_lib.qlinear_debug_dequant(fmt, _ptr(packed), _ptr(p0), _ptr(p1), _ptr(w), N, K,
                                       _stream(stream)), "qlinear_debug_dequant")
     return w
+
+
+def qlinear_dequant_fp16(fmt, packed, p0, p1, w, N, K, stream=None):
+    """Packed weights -> dense fp16 ``w[N, K]`` (see the C declaration for p0 / p1)."""
+    _check(_lib.qlinear_dequant_fp16(fmt, _ptr(packed), _ptr(p0), _ptr(p1), _ptr(w), N, K,
+                                     _stream(stream)), "qlinear_dequant_fp16")
+    return w
+
+
+def qlinear_prefill(fmt, x, packed, p0, p1, w_fp16, y, M, N, K, stream=None):
+    """``y[M, N] = x[M, K] @ w_fp16[N, K]^T`` after dequantizing into ``w_fp16``."""
+    _check(_lib.qlinear_prefill(fmt, _ptr(x), _ptr(packed), _ptr(p0), _ptr(p1), _ptr(w_fp16),
+                                _ptr(y), M, N, K, _stream(stream)), "qlinear_prefill")
+    return y

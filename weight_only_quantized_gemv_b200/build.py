@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libqlinear.so")
 
-SOURCES = ["qlinear.cu", "pack.cpp"]
+SOURCES = ["qlinear.cu", "dequant.cu", "pack.cpp"]
 HEADERS = ["kernels.cuh", "layout.h"]
 
 
@@ -34,7 +34,7 @@ def command(out: str = LIB, ptxas_verbose: bool = False) -> list:
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, s) for s in SOURCES]
-    cmd += ["-o", out, "-lgomp"]
+    cmd += ["-o", out, "-lgomp", "-ldl"]
     return cmd
 
 

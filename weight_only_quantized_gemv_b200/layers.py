@@ -13,7 +13,8 @@ import numpy as np
 import torch
 
 from . import (QL_FMT_LUT4, QL_FMT_W2, QL_FMT_W4, QL_FMT_W8, qlinear_debug_dequant,
-               qlinear_debug_unpack, qlinear_lut4, qlinear_pack, qlinear_pack_params,
+               qlinear_debug_unpack, qlinear_dequant_fp16, qlinear_lut4, qlinear_pack,
+               qlinear_pack_params, qlinear_prefill,
                qlinear_pack_tilecoo, qlinear_w2a16, qlinear_w4a16, qlinear_w4a16_outlier,
                qlinear_w8a16, qlinear_workspace_bytes)
 
@@ -75,6 +76,32 @@ class QuantLinear:
         else:
             _ENTRY[self.fmt](xv, self.qweight, self.p0, self.p1, yv, M, self.N, self.K,
                              self.workspace, stream)
+        return y
+
+    def dequant_fp16(self, w: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """The dense fp16 weights, ``w[N, K]`` (one row per output column)."""
+        if w is None:
+            w = torch.empty((self.N, self.K), dtype=torch.float16, device=self.device)
+        qlinear_dequant_fp16(self.fmt, self.qweight, self.p0, self.p1, w.view(torch.int16),
+                             self.N, self.K, stream)
+        return w
+
+    def prefill(self, x: torch.Tensor, y: Optional[torch.Tensor] = None,
+                w_fp16: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """y[M, N] = x[M, K] . W for any M: dequantize into ``w_fp16`` ([N, K] fp16, kept
+        by the layer when not given), then one dense GEMM.  Dense part only (no outliers)."""
+        if self.tile is not None:
+            raise ValueError("prefill covers the dense formats; the outlier layer has none")
+        M = x.shape[0]
+        if y is None:
+            y = torch.empty((M, self.N), dtype=torch.float16, device=self.device)
+        if w_fp16 is None:
+            if getattr(self, "_w_fp16", None) is None:
+                self._w_fp16 = torch.empty((self.N, self.K), dtype=torch.float16,
+                                           device=self.device)
+            w_fp16 = self._w_fp16
+        qlinear_prefill(self.fmt, x.view(torch.int16), self.qweight, self.p0, self.p1,
+                        w_fp16.view(torch.int16), y.view(torch.int16), M, self.N, self.K, stream)
         return y
 
     def debug_unpack(self, stream=None) -> torch.Tensor:
