@@ -221,6 +221,60 @@ ql_status qlinear_prefill(int fmt, const uint16_t* x, const void* packed, const 
                           ql_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Measured policy map and dispatcher.
+ * Source: ADAngel page (awesome-system-papers, OSDI'26), core method: an offline script
+ * times every candidate kernel with CUDA events over the (M, N, K) and bit-width
+ * combinations of a model and keeps the fastest in a table (the oracle policy map); at run
+ * time the dispatcher looks the shape and bit width up and calls that kernel.  The offline
+ * script here is the Python package's `tune` module; the table is host memory owned by the
+ * library (a copy of what qlinear_policy_set receives).
+ * ------------------------------------------------------------------------- */
+
+typedef enum {
+  QL_STRATEGY_GEMV = 0,    /* the fused GEMV (over 16-row slices of x when M > 16) */
+  QL_STRATEGY_PREFILL = 1  /* qlinear_prefill: dequantize to fp16, then one dense GEMM */
+} ql_strategy;
+
+typedef struct {
+  int fmt;             /* ql_format */
+  int N, K;            /* layer shape, matched exactly */
+  int m_lo, m_hi;      /* rows of x covered, inclusive, 1 <= m_lo <= m_hi */
+  int strategy;        /* ql_strategy */
+  int warps_per_unit;  /* GEMV: 0 = the planner's rule, else 1, 2 or 4 (honoured by the W4
+                          kernels at M <= 8; other kernels have one variant) */
+  int ctas;            /* GEMV: 0 = the planner's rule, else the grid size (clamped to the
+                          number of work units) */
+} ql_policy_entry;
+
+/* Install a policy table (copied; n = 0 clears it).  The first entry that covers a call
+ * decides it.  Entries apply to the plain formats, not to qlinear_w4a16_outlier.  A table
+ * changes grid sizes, so query qlinear_workspace_bytes after installing it.  Returns
+ * QL_ERR_UNSUPPORTED for an unknown format or strategy, QL_ERR_SHAPE for an invalid shape,
+ * M range, warps_per_unit or ctas (nothing is installed then). */
+ql_status qlinear_policy_set(const ql_policy_entry* entries, int n);
+
+/* Number of installed entries. */
+int qlinear_policy_size(void);
+
+/* The decision for (fmt, M, N, K): the covering table entry (*from_table = 1), else the
+ * built-in rule (*from_table = 0): the GEMV for M <= 64 with the planner's rules, prefill
+ * above; out->m_lo / m_hi give the rule's M range.  from_table may be NULL. */
+ql_status qlinear_policy_lookup(int fmt, int M, int N, int K, ql_policy_entry* out,
+                                int* from_table);
+
+/* y[M][N] = x[M][K] . dequant(W) for any M >= 1, by the policy's decision:
+ *   GEMV    : the format's GEMV entry (qlinear_w4a16 ...) on each 16-row slice of x / y in
+ *             turn, all with `workspace` (at least qlinear_workspace_bytes(fmt, min(M, 16), N,
+ *             K) bytes);
+ *   PREFILL : qlinear_prefill into w_fp16 (N * K fp16).  When w_fp16 is NULL the GEMV is
+ *             used instead.
+ * Arguments as in those entries (p0 / p1: scales / zeros, or lut16 / absmax for LUT4; group
+ * 128, LUT block 64).  Returns the first non-OK status of the calls it makes. */
+ql_status qlinear_matmul(int fmt, const uint16_t* x, const void* packed, const void* p0,
+                         const void* p1, uint16_t* y, int M, int N, int K, void* workspace,
+                         size_t workspace_bytes, uint16_t* w_fp16, ql_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Debug entries (device pointers, asynchronous).  They decode the packed layout
  * with the same fragment-extraction code the GEMV kernels use.
  *   qlinear_debug_unpack : codes uint8 [K][N] (canonical order, one code per byte)

@@ -37,6 +37,15 @@ _I = ctypes.c_int
 _SZ = ctypes.c_size_t
 
 
+class ql_policy_entry(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int), ("N", ctypes.c_int), ("K", ctypes.c_int),
+                ("m_lo", ctypes.c_int), ("m_hi", ctypes.c_int), ("strategy", ctypes.c_int),
+                ("warps_per_unit", ctypes.c_int), ("ctas", ctypes.c_int)]
+
+
+QL_STRATEGY_GEMV, QL_STRATEGY_PREFILL = 0, 1
+
+
 class ql_plan(ctypes.Structure):
     _fields_ = [("ctas", ctypes.c_int), ("warps", ctypes.c_int), ("tiles_per_warp", ctypes.c_int),
                 ("units", ctypes.c_longlong), ("m_bucket", ctypes.c_int),
@@ -63,6 +72,11 @@ _SIGS = {
     "qlinear_w4a16_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "qlinear_dequant_fp16": (_I, [_I, _P, _P, _P, _P, _I, _I, _P]),
     "qlinear_prefill": (_I, [_I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "qlinear_policy_set": (_I, [ctypes.POINTER(ql_policy_entry), _I]),
+    "qlinear_policy_size": (_I, []),
+    "qlinear_policy_lookup": (_I, [_I, _I, _I, _I, ctypes.POINTER(ql_policy_entry),
+                                   ctypes.POINTER(_I)]),
+    "qlinear_matmul": (_I, [_I, _P, _P, _P, _P, _P, _I, _I, _I, _P, _SZ, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -239,4 +253,52 @@ def qlinear_prefill(fmt, x, packed, p0, p1, w_fp16, y, M, N, K, stream=None):
     """``y[M, N] = x[M, K] @ w_fp16[N, K]^T`` after dequantizing into ``w_fp16``."""
     _check(_lib.qlinear_prefill(fmt, _ptr(x), _ptr(packed), _ptr(p0), _ptr(p1), _ptr(w_fp16),
                                 _ptr(y), M, N, K, _stream(stream)), "qlinear_prefill")
+    return y
+
+
+# ---------------------------------------------------------------------------
+# measured policy map and dispatcher
+
+
+_ENTRY_KEYS = ("fmt", "N", "K", "m_lo", "m_hi", "strategy", "warps_per_unit", "ctas")
+
+
+def qlinear_policy_set(entries) -> None:
+    """Install a policy table: a sequence of dicts (or ql_policy_entry) with the entry's
+    fields; an empty sequence clears it."""
+    arr = (ql_policy_entry * max(len(entries), 1))()
+    for i, e in enumerate(entries):
+        arr[i] = e if isinstance(e, ql_policy_entry) else \
+            ql_policy_entry(*[int(e.get(k, 0)) for k in _ENTRY_KEYS])
+    _check(_lib.qlinear_policy_set(arr, len(entries)), "qlinear_policy_set")
+
+
+def qlinear_policy_size() -> int:
+    return int(_lib.qlinear_policy_size())
+
+
+def qlinear_policy_lookup(fmt: int, M: int, N: int, K: int):
+    """(decision as a dict, whether it came from the table)."""
+    e = ql_policy_entry()
+    ft = _I(0)
+    _check(_lib.qlinear_policy_lookup(fmt, M, N, K, ctypes.byref(e), ctypes.byref(ft)),
+           "qlinear_policy_lookup")
+    return {k: getattr(e, k) for k in _ENTRY_KEYS}, bool(ft.value)
+
+
+def load_policy(path: str) -> int:
+    """Install the table of a JSON file written by the tune module; returns its size."""
+    import json
+    with open(path) as f:
+        table = json.load(f)
+    qlinear_policy_set(table["entries"])
+    return qlinear_policy_size()
+
+
+def qlinear_matmul(fmt, x, packed, p0, p1, y, M, N, K, workspace, w_fp16=None, stream=None):
+    """y[M, N] = x[M, K] . W for any M, by the policy map (GEMV slices or prefill)."""
+    st = _lib.qlinear_matmul(fmt, _ptr(x), _ptr(packed), _ptr(p0), _ptr(p1), _ptr(y), M, N, K,
+                             _ptr(workspace), workspace.numel() * workspace.element_size()
+                             if workspace is not None else 0, _ptr(w_fp16), _stream(stream))
+    _check(st, "qlinear_matmul")
     return y

@@ -16,8 +16,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libqlinear.so")
 
-SOURCES = ["qlinear.cu", "dequant.cu", "pack.cpp"]
-HEADERS = ["kernels.cuh", "layout.h"]
+SOURCES = ["qlinear.cu", "dequant.cu", "policy.cpp", "pack.cpp"]
+HEADERS = ["kernels.cuh", "layout.h", "policy.h"]
 
 
 def nvcc_path() -> str:

@@ -10,6 +10,7 @@
 #include <unordered_map>
 
 #include "kernels.cuh"
+#include "policy.h"
 #include "qlinear.h"
 
 using namespace qlayout;
@@ -153,6 +154,9 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
       small_m1 = true;
     }
   }
+  // a measured policy entry may fix the grid size and the warps per unit
+  const qpolicy::Choice pol = qpolicy::lookup(fmt, outl, M, N, K);
+  if (pol.ctas > 0) C = pol.ctas;
   // QLINEAR_MAX_CTAS forces the grid size (A/B runs, tests of the split-K fix-up)
   if (const char* cap = getenv("QLINEAR_MAX_CTAS")) {
     const long long v = atoll(cap);
@@ -173,6 +177,7 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
   if (fmt == kW4 && p->MT == 1 && !outl) {
     const long long per_cta = (p->U + C - 1) / C;
     int wpu = p->M1 ? 1 : per_cta <= 4 ? 4 : per_cta <= 24 ? 2 : 1;
+    if (pol.wpu > 0) wpu = pol.wpu;
     if (const char* w = getenv("QLINEAR_WPU")) {
       const int v = atoi(w);
       if (v == 1 || v == 2 || v == 4) wpu = v;

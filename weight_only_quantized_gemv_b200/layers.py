@@ -12,9 +12,10 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (QL_FMT_LUT4, QL_FMT_W2, QL_FMT_W4, QL_FMT_W8, qlinear_debug_dequant,
+from . import (QL_FMT_LUT4, QL_FMT_W2, QL_FMT_W4, QL_FMT_W8, QL_STRATEGY_PREFILL,
+               qlinear_debug_dequant, qlinear_policy_lookup,
                qlinear_debug_unpack, qlinear_dequant_fp16, qlinear_lut4, qlinear_pack,
-               qlinear_pack_params, qlinear_prefill,
+               qlinear_matmul, qlinear_pack_params, qlinear_prefill,
                qlinear_pack_tilecoo, qlinear_w2a16, qlinear_w4a16, qlinear_w4a16_outlier,
                qlinear_w8a16, qlinear_workspace_bytes)
 
@@ -102,6 +103,27 @@ class QuantLinear:
             w_fp16 = self._w_fp16
         qlinear_prefill(self.fmt, x.view(torch.int16), self.qweight, self.p0, self.p1,
                         w_fp16.view(torch.int16), y.view(torch.int16), M, self.N, self.K, stream)
+        return y
+
+    def matmul(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, stream=None,
+               allow_prefill: bool = True) -> torch.Tensor:
+        """y[M, N] = x[M, K] . W for any M, dispatched by the library's policy map (the fused
+        GEMV, over 16-row slices when M > 16, or the prefill path).  The layer's fp16 weight
+        buffer for prefill is allocated on the first call the policy sends to prefill."""
+        if self.tile is not None:
+            raise ValueError("the policy map covers the dense formats")
+        M = x.shape[0]
+        if y is None:
+            y = torch.empty((M, self.N), dtype=torch.float16, device=self.device)
+        wbuf = None
+        decision, _ = qlinear_policy_lookup(self.fmt, M, self.N, self.K)
+        if allow_prefill and decision["strategy"] == QL_STRATEGY_PREFILL:
+            if getattr(self, "_w_fp16", None) is None:
+                self._w_fp16 = torch.empty((self.N, self.K), dtype=torch.float16,
+                                           device=self.device)
+            wbuf = self._w_fp16.view(torch.int16)
+        qlinear_matmul(self.fmt, x.view(torch.int16), self.qweight, self.p0, self.p1,
+                       y.view(torch.int16), M, self.N, self.K, self.workspace, wbuf, stream)
         return y
 
     def debug_unpack(self, stream=None) -> torch.Tensor:

@@ -1,0 +1,190 @@
+"""Offline tuner that builds the measured policy map.
+
+    python -m weight_only_quantized_gemv_b200.tune --fmts w4,w2 \
+        --shapes 4096x4096,8192x28672 --M 1-16,32,64,128,512 --out policy.json
+
+Follows the ADAngel page (awesome-system-papers, OSDI'26, core method): for every
+(format, K x N layer, M) it runs each candidate of the strategy set through the library's
+dispatcher (`qlinear_matmul`), times it with CUDA events on the launching stream, and keeps
+the fastest.  Candidates:
+
+* the fused GEMV with the planner's rules;
+* for M <= 16, the GEMV with a fixed grid of 1, 2 or 3 CTAs per SM, and for W4 at
+  2 <= M <= 8 with 1, 2 or 4 warps per work unit;
+* the prefill path (dequantization to fp16 + dense GEMM).
+
+Each candidate is installed as a one-entry table, so the timed call is exactly the call a
+user makes.  Packed codes and parameters are random bytes of the right sizes, in enough
+copies (each with its own fp16 weight buffer) that every launch misses L2.  The measured
+M values become ranges: the choice at M_i covers (M_{i-1}, M_i], the last one every larger M.
+The JSON file holds the entries (for `load_policy`) and every timing.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+from typing import Dict, List, Sequence, Tuple
+
+FMT_CODES = {"w2": 2, "w4": 4, "w8": 8, "lut4": 16}
+M_MAX = 2 ** 31 - 1
+L2_BYTES = 126 * 2 ** 20
+
+Candidate = Tuple[int, int, int]  # (strategy, warps_per_unit, ctas)
+
+
+def parse_m_list(text: str) -> List[int]:
+    """'1-4,8,16' -> [1, 2, 3, 4, 8, 16] (sorted, unique)."""
+    out = set()
+    for part in text.split(","):
+        part = part.strip()
+        if not part:
+            continue
+        if "-" in part:
+            a, b = part.split("-")
+            out.update(range(int(a), int(b) + 1))
+        else:
+            out.add(int(part))
+    if not out or min(out) < 1:
+        raise ValueError(f"bad M list {text!r}")
+    return sorted(out)
+
+
+def parse_shapes(text: str) -> List[Tuple[int, int]]:
+    """'4096x4096,8192x28672' -> [(K, N), ...]."""
+    shapes = []
+    for part in text.split(","):
+        k, n = part.lower().split("x")
+        shapes.append((int(k), int(n)))
+    return shapes
+
+
+def candidates(fmt: int, M: int, sms: int) -> List[Candidate]:
+    c: List[Candidate] = [(0, 0, 0)]
+    if M <= 16:
+        c += [(0, 0, k * sms) for k in (1, 2, 3)]
+        if fmt == 4 and 2 <= M <= 8:
+            c += [(0, w, 0) for w in (1, 2, 4)]
+    c.append((1, 0, 0))
+    return c
+
+
+def build_entries(fmt: int, N: int, K: int, best: Dict[int, Candidate]) -> List[dict]:
+    """Turn the winner at each measured M into M ranges (merged when neighbours agree)."""
+    ms = sorted(best)
+    entries: List[dict] = []
+    lo = 1
+    for i, m in enumerate(ms):
+        hi = M_MAX if i == len(ms) - 1 else m
+        s, w, c = best[m]
+        if entries and (entries[-1]["strategy"], entries[-1]["warps_per_unit"],
+                        entries[-1]["ctas"]) == (s, w, c):
+            entries[-1]["m_hi"] = hi
+        else:
+            entries.append(dict(fmt=fmt, N=N, K=K, m_lo=lo, m_hi=hi, strategy=s,
+                                warps_per_unit=w, ctas=c))
+        lo = m + 1
+    return entries
+
+
+def tune_layer(fmt: int, K: int, N: int, m_list: Sequence[int], reps: int, log) -> Tuple[list, list]:
+    import torch
+
+    from . import (QL_FMT_LUT4, qlinear_matmul, qlinear_policy_set, qlinear_workspace_bytes)
+
+    dev = torch.device("cuda:0")
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    bits = 4 if fmt == QL_FMT_LUT4 else fmt
+    G = K // 128
+    per_copy = K * N * bits // 8 + 2 * N * K
+    copies = max(2, math.ceil(2 * L2_BYTES / per_copy))
+    gen = torch.Generator(device=dev).manual_seed(K * 7 + N)
+    q = [torch.randint(0, 256, (K * N * bits // 8,), dtype=torch.uint8, device=dev, generator=gen)
+         for _ in range(copies)]
+    if fmt == QL_FMT_LUT4:
+        p0 = [torch.linspace(-1, 1, 16, device=dev).half().view(torch.int16)] * copies
+        p1 = [torch.rand((K // 64) * N, device=dev, generator=gen) * 0.05 for _ in range(copies)]
+    else:
+        p0 = [(torch.rand(G * N, device=dev, generator=gen) * 0.01).half().view(torch.int16)
+              for _ in range(copies)]
+        p1 = [torch.randint(0, 1 << bits, (G * N,), device=dev, generator=gen).half()
+              .view(torch.int16) for _ in range(copies)]
+    wbuf = [torch.empty(N * K, dtype=torch.int16, device=dev) for _ in range(copies)]
+    Mmax = max(m_list)
+    x = torch.randn(Mmax, K, device=dev, generator=gen).half().view(torch.int16)
+    y = torch.empty(Mmax, N, device=dev, dtype=torch.int16)
+    ws_cache: Dict[int, torch.Tensor] = {}
+    timings, best = [], {}
+    for M in m_list:
+        results = []
+        for cand in candidates(fmt, M, sms):
+            s, w, c = cand
+            qlinear_policy_set([dict(fmt=fmt, N=N, K=K, m_lo=1, m_hi=M_MAX, strategy=s,
+                                     warps_per_unit=w, ctas=c)])
+            need = qlinear_workspace_bytes(fmt, min(M, 16), N, K)
+            if need not in ws_cache:
+                ws_cache[need] = torch.zeros(max(need, 256) // 4 + 64, dtype=torch.int32,
+                                             device=dev)
+            ws = ws_cache[need]
+
+            def call(i):
+                j = i % copies
+                qlinear_matmul(fmt, x, q[j], p0[j], p1[j], y, M, N, K, ws, wbuf[j])
+
+            for i in range(2 * copies):
+                call(i)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for i in range(reps):
+                call(i)
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / reps
+            results.append((us, cand))
+            timings.append(dict(fmt=fmt, K=K, N=N, M=M, strategy=s, warps_per_unit=w, ctas=c,
+                                us=round(us, 3)))
+        us, cand = min(results)
+        best[M] = cand
+        log(f"fmt={fmt} K={K} N={N} M={M}: best {cand} {us:.2f} us "
+            f"(rule {results[0][0]:.2f} us)")
+    qlinear_policy_set([])
+    del q, p0, p1, wbuf, x, y, ws_cache
+    torch.cuda.empty_cache()
+    return build_entries(fmt, N, K, best), timings
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--fmts", default="w4")
+    ap.add_argument("--shapes", default="4096x4096")
+    ap.add_argument("--M", default="1-16,24,32,48,64,96,128,256,512")
+    ap.add_argument("--reps", type=int, default=10)
+    ap.add_argument("--out", required=True)
+    a = ap.parse_args()
+    import sys
+
+    import torch
+
+    from . import qlinear_policy_set
+
+    torch.cuda.set_device(0)
+    m_list = parse_m_list(a.M)
+    entries, timings = [], []
+    for name in a.fmts.split(","):
+        for K, N in parse_shapes(a.shapes):
+            e, t = tune_layer(FMT_CODES[name], K, N, m_list, a.reps,
+                              lambda s: print(s, file=sys.stderr, flush=True))
+            entries += e
+            timings += t
+    qlinear_policy_set(entries)  # validates the table
+    qlinear_policy_set([])
+    props = torch.cuda.get_device_properties(0)
+    with open(a.out, "w") as f:
+        json.dump(dict(device=props.name, sms=props.multi_processor_count, M=m_list,
+                       entries=entries, timings=timings), f, indent=1)
+    print(json.dumps(dict(out=a.out, entries=len(entries), timings=len(timings))))
+
+
+if __name__ == "__main__":
+    main()
