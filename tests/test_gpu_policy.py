@@ -104,7 +104,9 @@ def test_larger_grid_needs_a_larger_workspace():
 def test_tuner_end_to_end_small_layer():
     K, N = 1024, 512
     m_list = [1, 4, 17, 80]
-    entries, timings = tune.tune_layer(4, K, N, m_list, reps=3, log=lambda s: None)
+    entries, timings, checks = tune.tune_layer(4, K, N, m_list, reps=3, log=lambda s: None,
+                                               validate=True)
+    assert [c["M"] for c in checks] == m_list and all(c["table_us"] > 0 for c in checks)
     assert len(timings) == sum(len(tune.candidates(4, m, torch.cuda.get_device_properties(0)
                                                    .multi_processor_count)) for m in m_list)
     assert all(t["us"] > 0 for t in timings)

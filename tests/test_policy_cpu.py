@@ -123,3 +123,35 @@ def test_build_entries_merges_ranges():
         d, t = ql.qlinear_policy_lookup(4, m, 512, 1024)
         assert t
         assert sum(1 for x in e if x["m_lo"] <= m <= x["m_hi"]) == 1
+
+
+def test_pick_keeps_the_rule_unless_beaten_by_the_margin():
+    rule = (100.0, (0, 0, 0))
+    assert tune.pick([rule, (99.0, (0, 2, 0)), (150.0, (1, 0, 0))], 0.02) == rule
+    assert tune.pick([rule, (97.0, (0, 2, 0))], 0.02) == (97.0, (0, 2, 0))
+    # the prefill strategy is taken whenever it is fastest (no margin)
+    assert tune.pick([rule, (99.5, (1, 0, 0))], 0.02) == (99.5, (1, 0, 0))
+
+
+def test_rule_choice_matches_the_library_rule():
+    for m in (1, 16, 64, 65, 512):
+        d, t = ql.qlinear_policy_lookup(4, m, 4096, 4096)
+        assert not t and tune.rule_choice(m) == (d["strategy"], d["warps_per_unit"], d["ctas"])
+
+
+def test_committed_b200_table_installs_and_covers_its_layers():
+    import json
+    with open(ql.default_policy_path()) as f:
+        table = json.load(f)
+    assert ql.load_policy() == len(table["entries"]) > 0
+    layers = {(e["fmt"], e["K"], e["N"]) for e in table["entries"]}
+    assert len(layers) == 24                       # 4 formats x 6 layers
+    for fmt, K, N in layers:
+        own = sorted((e["m_lo"], e["m_hi"]) for e in table["entries"]
+                     if (e["fmt"], e["K"], e["N"]) == (fmt, K, N))
+        assert own[0][0] == 1 and own[-1][1] == M_MAX
+        assert all(b[0] == a[1] + 1 for a, b in zip(own, own[1:]))   # contiguous, disjoint
+        for m in (1, 7, 16, 17, 64, 65, 4096):
+            assert ql.qlinear_policy_lookup(fmt, m, N, K)[1]
+    # the validation pairs were measured for every layer and M of the sweep
+    assert len(table["validation"]) == 24 * len(table["M"])

@@ -286,10 +286,17 @@ def qlinear_policy_lookup(fmt: int, M: int, N: int, K: int):
     return {k: getattr(e, k) for k in _ENTRY_KEYS}, bool(ft.value)
 
 
-def load_policy(path: str) -> int:
-    """Install the table of a JSON file written by the tune module; returns its size."""
+def default_policy_path() -> str:
+    """The table measured on B200 for the Llama-shaped layers (the package's policy_b200.json,
+    written by the tune module)."""
+    return os.path.join(_HERE, "policy_b200.json")
+
+
+def load_policy(path: Optional[str] = None) -> int:
+    """Install the table of a JSON file written by the tune module (default: the B200 table);
+    returns its size."""
     import json
-    with open(path) as f:
+    with open(path or default_policy_path()) as f:
         table = json.load(f)
     qlinear_policy_set(table["entries"])
     return qlinear_policy_size()
