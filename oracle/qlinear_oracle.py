@@ -26,6 +26,11 @@ Sources followed (page, section):
   values through a 16-entry table);
 * dense + sparse outlier decomposition ``y = x dequant(W_dense) + x W_out``:
   FlashQuant page, English abstract;
+* codebook (vector) quantization, m = 1 codebook of 2^b centroids of length v,
+  per-group normalization: ``w[k, n] = s[k // g, n] * C[code[k // v, n], k % v]``;
+  and its Psumbook evaluation ``p[j, i] = sum_t C[i, t] x[v j + t]``,
+  ``y[n] = sum_g s[g, n] sum_{j in g} p[j, code[j, n]]``: CodeGEMM page, method
+  (overall framework, key designs one and four);
 * stand-alone dequantization for prefill (fp16 weights written back to global
   memory, then an ordinary fp16 matmul): "Fast NF4 Dequantization Kernels"
   page, method section (technical framework: load codes, dequantize, write
@@ -210,6 +215,55 @@ def gemv_outlier(x: np.ndarray, qweight: np.ndarray, scales: np.ndarray, zeros: 
     dense = gemv_uniform(x, qweight, scales, zeros, bits, group, cols)
     sparse = x.astype(np.float64) @ tilecoo_to_dense(offsets, rc, vals, K, N, cols)
     return dense + sparse
+
+
+# ---------------------------------------------------------------------------
+# codebook quantization (CodeGEMM, m = 1): codes uint8 [K / v, N], codebook
+# [2^b, v], scales [K / g, N]
+
+
+def dequant_codebook(codes: np.ndarray, codebook: np.ndarray, scales: np.ndarray, v: int,
+                     group: int, cols: Optional[Sequence[int]] = None) -> np.ndarray:
+    """``w[k, n] = s[k // g, n] * C[code[k // v, n], k % v]`` in fp64."""
+    c = _col_select(codes, cols)
+    s = _col_select(scales, cols).astype(np.float64)
+    C = codebook.astype(np.float64)
+    K = c.shape[0] * v
+    k = np.arange(K)
+    return s[k // group, :] * C[c[k // v, :], (k % v)[:, None]]
+
+
+def gemv_codebook(x: np.ndarray, codes: np.ndarray, codebook: np.ndarray, scales: np.ndarray,
+                  v: int, group: int, cols: Optional[Sequence[int]] = None) -> np.ndarray:
+    """``y = x @ dequant(W)`` in fp64."""
+    return x.astype(np.float64) @ dequant_codebook(codes, codebook, scales, v, group, cols)
+
+
+def psumbook(x: np.ndarray, codebook: np.ndarray, v: int) -> np.ndarray:
+    """``P[m, j, i] = sum_t C[i, t] * x[m, v j + t]`` (fp64): every input slice of length v
+    against every centroid."""
+    xs = x.astype(np.float64)
+    M, K = xs.shape
+    return xs.reshape(M, K // v, v) @ codebook.astype(np.float64).T
+
+
+def gemv_codebook_psumbook(x: np.ndarray, codes: np.ndarray, codebook: np.ndarray,
+                           scales: np.ndarray, v: int, group: int,
+                           cols: Optional[Sequence[int]] = None) -> np.ndarray:
+    """The Psumbook evaluation: build P, look each code up, sum per group, scale, sum groups."""
+    P = psumbook(x, codebook, v)
+    c = _col_select(codes, cols).astype(np.int64)
+    s = _col_select(scales, cols).astype(np.float64)
+    M = P.shape[0]
+    J, N = c.shape
+    per = group // v
+    y = np.zeros((M, N), dtype=np.float64)
+    for g in range(J // per):
+        acc = np.zeros((M, N), dtype=np.float64)
+        for j in range(g * per, (g + 1) * per):
+            acc += P[:, j, :][:, c[j]]
+        y += s[g][None, :] * acc
+    return y
 
 
 # ---------------------------------------------------------------------------

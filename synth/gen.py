@@ -30,6 +30,17 @@ What is produced, and the recipe each follows
   min-max quantized over the non-outlier entries of each group, and each
   outlier's dense slot holds the group's zero code.
 
+* Codebook (the CodeGEMM page's m1v4g128 configuration: one codebook, vectors
+  of 4 weights along K, 8-bit codes, group normalization over 128 weights): a
+  256 x 4 fp16 codebook with entries from U(-1, 1).  The page's codebooks come
+  from K-means/AQLM calibration, which is training and out of scope; the
+  GEMV's arithmetic does not depend on how the codes were chosen.  By default
+  the codes are uniform random bytes and each (group, column) scale is
+  ``fp16(0.02 * (2.5 + U(0, 1)))`` (about the absmax of 128 N(0, 0.02)
+  draws); given weights ``w`` (small sizes), the scale is the group's fp16
+  absmax and each code is the centroid nearest to the normalized 4-vector
+  ``w / s`` (squared distance in fp64, lower index on a tie).
+
 None of these functions unpack codes, dequantize or multiply by x.
 """
 from __future__ import annotations
@@ -43,12 +54,15 @@ STREAM_W = 0
 STREAM_X = 1
 STREAM_OUTLIER = 2
 STREAM_LUT = 3
+STREAM_CB = 4
 
 GROUP = 128
 LUT_BLOCK = 64
 TILE = 128
 OUTLIER_FRACTION = 0.005
 OUTLIER_SCALE = 10.0
+CB_VEC = 4          # weights per codebook vector (along K)
+CB_ENTRIES = 256    # 8-bit codes
 
 
 def workload_seed(workload: int, layer: int) -> int:
@@ -283,3 +297,40 @@ WORKLOADS = {
     3: dict(kind="lut4", shapes=[(8192, 28672), (28672, 8192)], M=[1]),
     4: dict(kind="outlier", shapes=[(4096, 14336), (8192, 28672)], M=[1, 2, 4, 8, 16]),
 }
+
+
+# ---------------------------------------------------------------------------
+# codebook (vector) quantization, m = 1 codebook, v = 4, b = 8
+
+
+@dataclasses.dataclass
+class CodebookLayer:
+    K: int
+    N: int
+    group: int
+    codebook: np.ndarray   # fp16[256, 4]
+    codes: np.ndarray      # uint8[K / 4, N]: code of the 4-vector (4j .. 4j + 3, n)
+    scales: np.ndarray     # fp16[K / group, N]
+
+
+def codebook_layer(seed: int, K: int, N: int, group: int = GROUP,
+                   w: Optional[np.ndarray] = None) -> CodebookLayer:
+    r = rng(seed, STREAM_CB)
+    codebook = r.uniform(-1.0, 1.0, size=(CB_ENTRIES, CB_VEC)).astype(np.float16)
+    if w is None:
+        codes = r.integers(0, CB_ENTRIES, size=(K // CB_VEC, N), dtype=np.uint8)
+        scales = (0.02 * (2.5 + r.uniform(0.0, 1.0, size=(K // group, N)))).astype(np.float16)
+        return CodebookLayer(K, N, group, codebook, codes, scales)
+    G = K // group
+    wg = w.astype(np.float64).reshape(G, group, N)
+    scales = np.abs(wg).max(axis=1).astype(np.float16)
+    s = scales.astype(np.float64)
+    ok = s > 0
+    u = wg / np.where(ok, s, 1.0)[:, None, :]                      # [G, group, N]
+    vec = u.reshape(G, group // CB_VEC, CB_VEC, N).transpose(0, 1, 3, 2).reshape(-1, CB_VEC)
+    c = codebook.astype(np.float64)
+    d = ((vec[:, None, :] - c[None, :, :]) ** 2).sum(axis=2)        # [vectors, 256]
+    idx = d.argmin(axis=1).astype(np.uint8)                         # first minimum on a tie
+    codes = idx.reshape(G, group // CB_VEC, N).reshape(K // CB_VEC, N)
+    codes = np.where(np.repeat(ok, group // CB_VEC, axis=0), codes, np.uint8(0))
+    return CodebookLayer(K, N, group, codebook, codes.astype(np.uint8), scales)
