@@ -221,6 +221,45 @@ ql_status qlinear_prefill(int fmt, const uint16_t* x, const void* packed, const 
                           ql_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Codebook GEMV with a Psumbook.  Source: CodeGEMM page (NeurIPS 2025 notes), method:
+ * overall framework (build the Psumbook, look codes up, accumulate), key design one
+ * (precomputed centroid . input partial sums kept in shared memory instead of the
+ * codebook), key design four (group normalization); configuration m1v4g128 (one codebook,
+ * 4-weight vectors, 8-bit codes: 2 bits per weight plus one fp16 scale per 128).
+ *
+ *   w[k][n] = s[k / 128][n] * C[code[k / 4][n]][k % 4]
+ *   y[m][n] = sum_g s[g][n] * sum_{j in g} P[m][j][code[j][n]],  P[m][j][i] = sum_t C[i][t] x[m][4j + t]
+ *
+ * Canonical layouts (host): codes uint8 [K / 4][N] (code of the 4-vector k = 4j .. 4j + 3
+ * of column n); scales fp16 [K / 128][N]; codebook fp16 [256][4] (used as is by the GEMV).
+ * Shapes: N % 32 == 0, K % 128 == 0, 1 <= M <= 4.  The Psumbook entries and every sum are
+ * fp32; y is rounded once to fp16.
+ * ------------------------------------------------------------------------- */
+
+/* Reorder canonical codes into the kernel layout: 32-column tiles by 128-k groups, each
+ * (tile, group) chunk 1024 bytes in which lane l's 32 codes form two 16-byte quads.  Host
+ * buffers of K / 4 * N bytes. */
+ql_status qlinear_pack_codebook(const uint8_t* codes, uint8_t* packed, int N, int K);
+
+/* Reorder canonical scales into chunk order, fp16 [tile][group][lane].  Host buffers of
+ * K / 128 * N fp16. */
+ql_status qlinear_pack_codebook_scales(const uint16_t* scales, uint16_t* packed, int N, int K);
+
+/* Workspace bytes for qlinear_codebook (per-tile arrival counters and fp32 partial sums of
+ * the K ranges); 0 for invalid shapes or without a device.  Zero-fill it once before its
+ * first use; every completed call leaves the counters at zero. */
+size_t qlinear_codebook_workspace_bytes(int M, int N, int K);
+
+/* y[M][N] = x[M][K] . W.  Device pointers: x fp16 (2-byte aligned), codes and scales as
+ * packed above (16- and 2-byte aligned), codebook fp16 [256][4] (8-byte aligned), y fp16.
+ * The workspace (16-byte aligned) is needed when the K range is split across CTAs (any
+ * K > 256 at M = 1, K > 128 otherwise).  Asynchronous on `stream`; results are bit-for-bit
+ * reproducible (partials are summed in a fixed order). */
+ql_status qlinear_codebook(const uint16_t* x, const uint8_t* codes, const uint16_t* scales,
+                           const uint16_t* codebook, uint16_t* y, int M, int N, int K,
+                           void* workspace, size_t workspace_bytes, ql_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Measured policy map and dispatcher.
  * Source: ADAngel page (awesome-system-papers, OSDI'26), core method: an offline script
  * times every candidate kernel with CUDA events over the (M, N, K) and bit-width

@@ -164,3 +164,40 @@ def test_prefill_entries_validate_before_any_device_work(ql):
     assert pf(4, a, a, a, a, a, a, 64, 120, 128, None) == 2
     assert pf(4, a + 1, a, a, a, a, a, 64, 128, 128, None) == 3
     assert pf(4, a, a, a, a, a + 2, a, 64, 128, 128, None) == 3
+
+
+def test_codebook_packers_and_checks(ql):
+    K, N = 384, 96
+    rs = np.random.default_rng(77)
+    codes = rs.integers(0, 256, size=(K // 4, N), dtype=np.uint8)
+    packed = ql.qlinear_pack_codebook(codes, N, K)
+    assert packed.nbytes == codes.nbytes
+    assert np.array_equal(np.sort(packed), np.sort(codes.reshape(-1)))
+    # one marked code lands at the documented position: chunk (tile, group), lane, quad
+    one = np.zeros_like(codes)
+    j, n = 37, 70                   # group 1, slice 5; tile 2, lane 6
+    one[j, n] = 1
+    p1 = ql.qlinear_pack_codebook(one, N, K)
+    G = K // 128
+    ch = (n // 32) * G + j // 32
+    jj, lane = j % 32, n % 32
+    assert np.flatnonzero(p1).tolist() == [ch * 1024 + ((jj // 16) * 32 + lane) * 16 + jj % 16]
+    s = np.arange((K // 128) * N, dtype=np.uint16).reshape(K // 128, N)
+    ps = ql.qlinear_pack_codebook_scales(s, N, K)
+    assert ps[((n // 32) * G + 2) * 32 + lane] == s[2, n]
+    assert sorted(ps.tolist()) == sorted(s.reshape(-1).tolist())
+    lib = ql._lib
+    buf = np.zeros(64, dtype=np.uint8)
+    assert lib.qlinear_pack_codebook(None, buf.ctypes.data, 32, 128) == 1
+    assert lib.qlinear_pack_codebook(buf.ctypes.data, buf.ctypes.data, 48, 128) == 2
+    a = 1 << 20
+    cb = lib.qlinear_codebook
+    assert cb(None, a, a, a, a, 1, 128, 128, a, 1 << 20, None) == 1
+    assert cb(a, a, a, a, a, 5, 128, 128, a, 1 << 20, None) == 2
+    assert cb(a, a, a, a, a, 0, 128, 128, a, 1 << 20, None) == 2
+    assert cb(a, a, a, a, a, 1, 48, 128, a, 1 << 20, None) == 2
+    assert cb(a, a, a, a, a, 1, 128, 100, a, 1 << 20, None) == 2
+    assert cb(a, a + 8, a, a, a, 1, 128, 128, a, 1 << 20, None) == 3
+    assert cb(a, a, a, a + 4, a, 1, 128, 128, a, 1 << 20, None) == 3
+    assert cb(a + 1, a, a, a, a, 1, 128, 128, a, 1 << 20, None) == 3
+    assert lib.qlinear_codebook_workspace_bytes(5, 128, 128) == 0

@@ -77,6 +77,10 @@ _SIGS = {
     "qlinear_policy_lookup": (_I, [_I, _I, _I, _I, ctypes.POINTER(ql_policy_entry),
                                    ctypes.POINTER(_I)]),
     "qlinear_matmul": (_I, [_I, _P, _P, _P, _P, _P, _I, _I, _I, _P, _SZ, _P, _P]),
+    "qlinear_pack_codebook": (_I, [_P, _P, _I, _I]),
+    "qlinear_pack_codebook_scales": (_I, [_P, _P, _I, _I]),
+    "qlinear_codebook_workspace_bytes": (_SZ, [_I, _I, _I]),
+    "qlinear_codebook": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _SZ, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -308,4 +312,39 @@ def qlinear_matmul(fmt, x, packed, p0, p1, y, M, N, K, workspace, w_fp16=None, s
                              _ptr(workspace), workspace.numel() * workspace.element_size()
                              if workspace is not None else 0, _ptr(w_fp16), _stream(stream))
     _check(st, "qlinear_matmul")
+    return y
+
+
+# ---------------------------------------------------------------------------
+# codebook GEMV (Psumbook)
+
+
+def qlinear_pack_codebook(codes: np.ndarray, N: int, K: int) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    if codes.size != K // 4 * N:
+        raise QLinearError(2, "qlinear_pack_codebook")
+    out = np.empty(codes.size, dtype=np.uint8)
+    _check(_lib.qlinear_pack_codebook(_np_ptr(codes), _np_ptr(out), N, K), "qlinear_pack_codebook")
+    return out
+
+
+def qlinear_pack_codebook_scales(scales: np.ndarray, N: int, K: int) -> np.ndarray:
+    scales = np.ascontiguousarray(scales).view(np.uint16)
+    if scales.size != K // 128 * N:
+        raise QLinearError(2, "qlinear_pack_codebook_scales")
+    out = np.empty(scales.size, dtype=np.uint16)
+    _check(_lib.qlinear_pack_codebook_scales(_np_ptr(scales), _np_ptr(out), N, K),
+           "qlinear_pack_codebook_scales")
+    return out
+
+
+def qlinear_codebook_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_lib.qlinear_codebook_workspace_bytes(M, N, K))
+
+
+def qlinear_codebook(x, codes, scales, codebook, y, M, N, K, workspace, stream=None):
+    st = _lib.qlinear_codebook(_ptr(x), _ptr(codes), _ptr(scales), _ptr(codebook), _ptr(y), M, N,
+                               K, _ptr(workspace), workspace.numel() * workspace.element_size()
+                               if workspace is not None else 0, _stream(stream))
+    _check(st, "qlinear_codebook")
     return y

@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libqlinear.so")
 
-SOURCES = ["qlinear.cu", "dequant.cu", "policy.cpp", "pack.cpp"]
+SOURCES = ["qlinear.cu", "dequant.cu", "codebook.cu", "policy.cpp", "pack.cpp"]
 HEADERS = ["kernels.cuh", "layout.h", "policy.h"]
 
 
