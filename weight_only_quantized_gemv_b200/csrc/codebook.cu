@@ -16,11 +16,14 @@
 // + j % 16, so one warp reads a chunk with two coalesced 512-byte loads.  Scales follow the
 // chunk order: fp16 [T][g][lane].
 //
-// Work split: the groups are cut into R ranges of GC groups (the Psumbook of a range fits
-// in shared memory), the tiles into P partitions; CTA (r, p) builds range r's Psumbook
-// once and streams the chunks of its tiles.  Each warp leaves one fp32 partial per (row,
-// column) and range; the last warp to arrive at a tile sums the R partials in range order
-// (deterministic) and stores fp16.
+// Work split: K is cut into R ranges of SL 4-slices (64 at M = 1, 32 at M = 2, 16 at
+// M = 3, 4: the Psumbook of a range, SL x 256 entries x the rows padded to 1, 2 or 4, is
+// 64 KB), the tiles into P partitions; CTA (r, p) builds range r's Psumbook once and
+// streams the codes of its tiles, each warp loading the next tile's codes before it works
+// through the current one.  Each warp leaves one fp32 partial per (row, column) and range
+// for each of its tiles, publishes them once at its end (one fence, one arrival per tile),
+// and the warp that arrives last at a tile sums the R partials in range order
+// (deterministic) and stores fp16.  A group's scale multiplies the sum of each 16 lookups of that group.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -61,128 +64,198 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return v;
 }
 
-template <int MR, int GC>
-constexpr int cb_smem_bytes() {
-  return MR * GC * kCbSlices * kCbEntries * 4 + MR * GC * kCbGroup * 4;
+// Rows of x padded to a vector width: the Psumbook keeps the MP rows of one (slice, code)
+// entry side by side, so one 4-, 8- or 16-byte lookup serves every row.
+template <int MR>
+__host__ __device__ constexpr int cb_mp() { return MR == 1 ? 1 : MR == 2 ? 2 : 4; }
+
+// Slices (4-vectors along K) per K range: the Psumbook of a range is SL x 256 x MP fp32 =
+// 64 KB for every M, three CTAs per SM.
+template <int MR>
+__host__ __device__ constexpr int cb_sl() { return MR == 1 ? 64 : MR == 2 ? 32 : 16; }
+
+template <int MR>
+__host__ __device__ constexpr int cb_smem_bytes() {
+  return cb_sl<MR>() * kCbEntries * cb_mp<MR>() * 4 + MR * cb_sl<MR>() * kCbVec * 4;
 }
 
-template <int MR, int GC>
-__global__ void __launch_bounds__(kCbThreads, (MR * GC <= 2) ? 3 : 1)
-    codebook_psum_kernel(const CbParams P) {
+template <int MP>
+struct CbVecT;
+template <> struct CbVecT<1> { using T = float; };
+template <> struct CbVecT<2> { using T = float2; };
+template <> struct CbVecT<4> { using T = float4; };
+
+__device__ __forceinline__ void cb_add(float (&a)[4], float v) { a[0] += v; }
+__device__ __forceinline__ void cb_add(float (&a)[4], float2 v) { a[0] += v.x; a[1] += v.y; }
+__device__ __forceinline__ void cb_add(float (&a)[4], float4 v) {
+  a[0] += v.x; a[1] += v.y; a[2] += v.z; a[3] += v.w;
+}
+
+template <int MR>
+__global__ void __launch_bounds__(kCbThreads, 3) codebook_psum_kernel(const CbParams P) {
+  constexpr int MP = cb_mp<MR>(), SL = cb_sl<MR>(), NQ = SL / 16;
+  using VecT = typename CbVecT<MP>::T;
   extern __shared__ __align__(16) float cb_smem[];
-  float* psum = cb_smem;                                         // [MR][GC][32][256]
-  float* xs = cb_smem + MR * GC * kCbSlices * kCbEntries;        // [MR][GC * 128]
+  float* psum = cb_smem;                               // [SL][256][MP]
+  float* xs = cb_smem + SL * kCbEntries * MP;          // [MR][SL * 4]
   const int r = blockIdx.x % P.R, part = blockIdx.x / P.R;
-  const int g0 = r * GC;
-  const int gc = min(GC, P.G - g0);
+  const int J = P.K / kCbVec;                          // slices in K
+  const int j0 = r * SL;
+  const int nsl = min(SL, J - j0);                     // a multiple of 16 (K % 128 == 0)
   const int tid = threadIdx.x;
 
-  // -- Psumbook of groups g0 .. g0 + gc - 1 -------------------------------------------
-  for (int i = tid; i < MR * gc * kCbGroup; i += kCbThreads) {
-    const int m = i / (gc * kCbGroup), e = i - m * gc * kCbGroup;
-    xs[m * GC * kCbGroup + e] = __half2float(P.x[(size_t)m * P.K + (size_t)g0 * kCbGroup + e]);
+  // -- Psumbook of slices j0 .. j0 + nsl - 1 ---------------------------------------------
+  for (int i = tid; i < MR * nsl * kCbVec; i += kCbThreads) {
+    const int m = i / (nsl * kCbVec), e = i - m * nsl * kCbVec;
+    xs[m * SL * kCbVec + e] = __half2float(P.x[(size_t)m * P.K + (size_t)j0 * kCbVec + e]);
   }
   __syncthreads();
   {
     const uint2 cw = reinterpret_cast<const uint2*>(P.codebook)[tid];  // centroid tid
     const float2 c01 = __half22float2(*reinterpret_cast<const __half2*>(&cw.x));
     const float2 c23 = __half22float2(*reinterpret_cast<const __half2*>(&cw.y));
+#pragma unroll 4
+    for (int j = 0; j < nsl; ++j) {
+      float pv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int m = 0; m < MR; ++m)
-      for (int gg = 0; gg < gc; ++gg)
-#pragma unroll 8
-        for (int j = 0; j < kCbSlices; ++j) {
-          const float4 xv = *reinterpret_cast<const float4*>(xs + m * GC * kCbGroup + gg * kCbGroup + 4 * j);
-          const float p = fmaf(c23.y, xv.w, fmaf(c23.x, xv.z, fmaf(c01.y, xv.y, c01.x * xv.x)));
-          psum[((m * GC + gg) * kCbSlices + j) * kCbEntries + tid] = p;
-        }
+      for (int m = 0; m < MR; ++m) {
+        const float4 xv = *reinterpret_cast<const float4*>(xs + m * SL * kCbVec + 4 * j);
+        pv[m] = fmaf(c23.y, xv.w, fmaf(c23.x, xv.z, fmaf(c01.y, xv.y, c01.x * xv.x)));
+      }
+      float* dst = psum + ((size_t)j * kCbEntries + tid) * MP;
+      if constexpr (MP == 1) dst[0] = pv[0];
+      else if constexpr (MP == 2) *reinterpret_cast<float2*>(dst) = make_float2(pv[0], pv[1]);
+      else *reinterpret_cast<float4*>(dst) = make_float4(pv[0], pv[1], pv[2], pv[3]);
+    }
   }
   __syncthreads();
 
-  // -- stream the tiles: one lookup and one add per code ---------------------------------
+  // -- stream the tiles: one lookup and one add per code, codes prefetched a tile ahead ---
   const int warp = tid >> 5, lane = tid & 31;
-  const uint32_t psum_s = (uint32_t)__cvta_generic_to_shared(psum);
-  for (int T = part * (kCbThreads / 32) + warp; T < P.ntiles; T += P.P * (kCbThreads / 32)) {
-    float acc[MR];
+  const int stride = P.P * (kCbThreads / 32);
+  const int nq = nsl / 16;
+  // quad qi of the range: slices j0 + 16 qi .. + 15, i.e. half (j0 / 16 + qi) % 2 of group
+  // (j0 / 16 + qi) / 2
+  auto load = [&](int T, uint4 (&cq)[NQ], float (&sc)[NQ]) {
 #pragma unroll
-    for (int m = 0; m < MR; ++m) acc[m] = 0.f;
-    uint4 cq[GC][2];
-    float sc[GC];
-#pragma unroll
-    for (int gg = 0; gg < GC; ++gg) {
-      if (gg < gc) {
-        const size_t ch = (size_t)T * P.G + g0 + gg;
-        const uint8_t* src = P.codes + ch * (kCbTile * kCbSlices);
-        cq[gg][0] = ldg_stream(src + (size_t)lane * 16);
-        cq[gg][1] = ldg_stream(src + (size_t)(32 + lane) * 16);
-        sc[gg] = __half2float(P.scales[ch * kCbTile + lane]);
+    for (int qi = 0; qi < NQ; ++qi) {
+      if (qi < nq) {
+        const int b16 = j0 / 16 + qi;
+        const size_t ch = (size_t)T * P.G + (b16 >> 1);
+        cq[qi] = ldg_stream(P.codes + ch * (kCbTile * kCbSlices) + (size_t)((b16 & 1) * 32 + lane) * 16);
+        sc[qi] = __half2float(P.scales[ch * kCbTile + lane]);
       }
     }
+  };
+  int T = part * (kCbThreads / 32) + warp;
+  uint4 cq[NQ];
+  float sc[NQ];
+  if (T < P.ntiles) load(T, cq, sc);
+  while (T < P.ntiles) {
+    const int Tn = T + stride;
+    uint4 nq4[NQ];
+    float nsc[NQ];
+    if (Tn < P.ntiles) load(Tn, nq4, nsc);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int gg = 0; gg < GC; ++gg) {
-      if (gg >= gc) break;
-      const uint32_t w[8] = {cq[gg][0].x, cq[gg][0].y, cq[gg][0].z, cq[gg][0].w,
-                             cq[gg][1].x, cq[gg][1].y, cq[gg][1].z, cq[gg][1].w};
+    for (int qi = 0; qi < NQ; ++qi) {
+      if (qi >= nq) break;
+      const uint32_t w[4] = {cq[qi].x, cq[qi].y, cq[qi].z, cq[qi].w};
+      const VecT* tab = reinterpret_cast<const VecT*>(psum) + qi * 16 * kCbEntries;
+      float s4[4][4] = {};
 #pragma unroll
-      for (int m = 0; m < MR; ++m) {
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint32_t base = psum_s + (uint32_t)((m * GC + gg) * kCbSlices * kCbEntries * 4);
-#pragma unroll
-        for (int j = 0; j < kCbSlices; ++j) {
-          const uint32_t code = (w[j >> 2] >> (8 * (j & 3))) & 0xFFu;
-          float v;
-          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v)
-                       : "r"(base + (uint32_t)(j * kCbEntries * 4) + code * 4u));
-          s4[j & 3] += v;
-        }
-        acc[m] = fmaf(sc[gg], (s4[0] + s4[1]) + (s4[2] + s4[3]), acc[m]);
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t code = __byte_perm(w[j >> 2], 0u, 0x4440u | (uint32_t)(j & 3));
+        cb_add(s4[j & 3], tab[j * kCbEntries + code]);
       }
+#pragma unroll
+      for (int m = 0; m < MR; ++m)
+        acc[m] = fmaf(sc[qi], (s4[0][m] + s4[1][m]) + (s4[2][m] + s4[3][m]), acc[m]);
     }
     const int n = T * kCbTile + lane;
     if (P.R == 1) {
 #pragma unroll
       for (int m = 0; m < MR; ++m) P.y[(size_t)m * P.N + n] = __float2half_rn(acc[m]);
-      continue;
+    } else {
+#pragma unroll
+      for (int m = 0; m < MR; ++m) P.partials[((size_t)r * MR + m) * P.N + n] = acc[m];
     }
 #pragma unroll
-    for (int m = 0; m < MR; ++m) P.partials[((size_t)r * MR + m) * P.N + n] = acc[m];
-    __threadfence();
-    __syncwarp();
-    uint32_t old = 0;
-    if (lane == 0) {
-      asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(P.counters + T) : "memory");
+    for (int qi = 0; qi < NQ; ++qi) {
+      cq[qi] = nq4[qi];
+      sc[qi] = nsc[qi];
     }
-    old = __shfl_sync(0xffffffffu, old, 0);
-    if (old == (uint32_t)(P.R - 1)) {  // last range to arrive: sum all R in range order
-      __threadfence();
+    T = Tn;
+  }
+  if (P.R == 1) return;
+
+  // -- publish this warp's partials once, then finish the tiles it reached last ---------
+  // (a fence per tile would wait for the prefetched codes of the next tile every time)
+  const int T0 = part * (kCbThreads / 32) + warp;
+  const int cnt = T0 < P.ntiles ? (P.ntiles - 1 - T0) / stride + 1 : 0;
+  __threadfence();
+  __syncwarp();
+  for (int b = 0; b < cnt; b += 32) {
+    bool last = false;
+    if (b + lane < cnt) {
+      uint32_t old;
+      asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old)
+                   : "l"(P.counters + T0 + (b + lane) * stride) : "memory");
+      last = old == (uint32_t)(P.R - 1);
+    }
+    uint32_t mask = __ballot_sync(0xffffffffu, last);
+    if (mask) __threadfence();
+    while (mask) {  // tiles whose every range has arrived: sum the R partials in range order
+      const int i = __ffs(mask) - 1;
+      mask &= mask - 1;
+      const int Tl = T0 + (b + i) * stride;
+      const int nl = Tl * kCbTile + lane;
+      // loads issued eight ranges at a time (independent, so their latencies overlap),
+      // added in range order
+      float t[MR];
 #pragma unroll
-      for (int m = 0; m < MR; ++m) {
-        float t = 0.f;
-        for (int rr = 0; rr < P.R; ++rr) t += __ldcg(P.partials + ((size_t)rr * MR + m) * P.N + n);
-        P.y[(size_t)m * P.N + n] = __float2half_rn(t);
+      for (int m = 0; m < MR; ++m) t[m] = 0.f;
+      const float* pp = P.partials + nl;
+      const size_t rs = (size_t)MR * P.N;
+      int rr = 0;
+      for (; rr + 8 <= P.R; rr += 8) {
+        float v[8][MR];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+          for (int m = 0; m < MR; ++m) v[u][m] = __ldcg(pp + (size_t)(rr + u) * rs + (size_t)m * P.N);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+          for (int m = 0; m < MR; ++m) t[m] += v[u][m];
       }
-      if (lane == 0) P.counters[T] = 0u;  // ready for the next call
+      for (; rr < P.R; ++rr)
+#pragma unroll
+        for (int m = 0; m < MR; ++m) t[m] += __ldcg(pp + (size_t)rr * rs + (size_t)m * P.N);
+#pragma unroll
+      for (int m = 0; m < MR; ++m) P.y[(size_t)m * P.N + nl] = __float2half_rn(t[m]);
+      if (lane == 0) P.counters[Tl] = 0u;  // ready for the next call
     }
   }
 }
 
 struct CbKernel {
   const void* fn;
-  int smem, GC;
+  int smem, SL;
 };
 
-template <int MR, int GC>
+template <int MR>
 CbKernel cb_kernel() {
-  return CbKernel{reinterpret_cast<const void*>(codebook_psum_kernel<MR, GC>), cb_smem_bytes<MR, GC>(),
-                  GC};
+  return CbKernel{reinterpret_cast<const void*>(codebook_psum_kernel<MR>), cb_smem_bytes<MR>(),
+                  cb_sl<MR>()};
 }
 
 CbKernel select_cb(int M) {
   switch (M) {
-    case 1: return cb_kernel<1, 2>();
-    case 2: return cb_kernel<2, 1>();
-    case 3: return cb_kernel<3, 1>();
-    default: return cb_kernel<4, 1>();
+    case 1: return cb_kernel<1>();
+    case 2: return cb_kernel<2>();
+    case 3: return cb_kernel<3>();
+    default: return cb_kernel<4>();
   }
 }
 
@@ -219,7 +292,8 @@ cudaError_t cb_plan(int M, int N, int K, CbPlan* p) {
   }
   p->G = K / kCbGroup;
   p->ntiles = N / kCbTile;
-  p->R = (p->G + p->k.GC - 1) / p->k.GC;
+  const int J = K / kCbVec;
+  p->R = (J + p->k.SL - 1) / p->k.SL;
   const long long slots = (long long)sms * occ;
   const long long tile_rows = (p->ntiles + kCbThreads / 32 - 1) / (kCbThreads / 32);
   long long parts = slots / p->R;
