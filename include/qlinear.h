@@ -33,6 +33,12 @@
  *     anything is enqueued; QL_ERR_CUDA reports a launch failure (cudaGetLastError).
  *   - Shapes: K % 128 == 0, N % 16 == 0, 1 <= M <= 16; the outlier variant also needs
  *     N % 128 == 0.  All 2-bit shapes with K % 128 == 0 are accepted.
+ *   - Group sizes (W2 / W4 / W8 entries, `group` argument): 128; 64 and 32 (finer groups,
+ *     parameters packed by qlinear_pack_params_grouped; QFactory page, "问题与动机" and
+ *     Differentiated Qtile Scheduling: fine-grained groups, their parameters reused from
+ *     registers); K (per-channel: one scale and zero per column, repeated per 128-k unit by
+ *     qlinear_pack_params_grouped, then read like group 128).  LUT4 (block 64), the outlier
+ *     variant and qlinear_w4a16_noalloc take their fixed block / group only.
  *   - Calls are thread-safe; two calls that share one workspace must not overlap in time
  *     (issue them on one stream).
  *
@@ -98,6 +104,18 @@ ql_status qlinear_pack(int fmt, const void* canonical, void* packed, int N, int 
  * scales and again for the zeros of W2/W4/W8 (fp16 [K/128][N]), or for the absmax of
  * LUT4 (fp32 [K/64][N]).  Host buffers of qlinear_params_bytes(). */
 ql_status qlinear_pack_params(int fmt, const void* canonical, void* packed, int N, int K);
+
+/* Bytes of packed scales (or zeros) for group size `group` of W2 / W4 / W8: K / 128 * NS * N
+ * fp16, NS = 128 / group for groups 32 and 64, 1 for 128 and for per-channel (group = K);
+ * 0 for other formats, groups or shapes. */
+size_t qlinear_params_bytes_grouped(int fmt, int group, int N, int K);
+
+/* Reorder one canonical parameter array (fp16 [K / group][N]; [1][N] for group = K) into
+ * the kernel layout for that group size: per chunk, per sub-group, for gi = 0..7 the pair
+ * of columns (gi, gi + 8).  Per-channel parameters are repeated in every 128-k unit.  Host
+ * buffers; the output holds qlinear_params_bytes_grouped() bytes. */
+ql_status qlinear_pack_params_grouped(int fmt, int group, const void* canonical, void* packed,
+                                      int N, int K);
 
 /* Reorder canonical Tile-COO (tiles numbered t = kt * (N/128) + nt) into the order the
  * fused outlier kernel walks them, t' = nt * (K/128) + kt, so that the outliers of one run

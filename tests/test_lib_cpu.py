@@ -122,7 +122,7 @@ def test_hot_path_validates_before_any_device_work(ql):
     assert call(x=None) == 1
     assert call(y=None) == 1
     assert call(M=0) == 2 and call(M=17) == 2
-    assert call(N=24) == 2 and call(K=100) == 2 and call(g=64) == 2
+    assert call(N=24) == 2 and call(K=100) == 2 and call(g=96) == 2 and call(g=256) == 2
     assert call(x=a + 2) == 3 and call(q=a + 16) == 3 and call(s=a + 2) == 3
     # scales and zeros are bulk-copied: 16-byte aligned sources only
     assert call(s=a + 4) == 3 and call(z=a + 8) == 3
@@ -201,3 +201,33 @@ def test_codebook_packers_and_checks(ql):
     assert cb(a, a, a, a + 4, a, 1, 128, 128, a, 1 << 20, None) == 3
     assert cb(a + 1, a, a, a, a, 1, 128, 128, a, 1 << 20, None) == 3
     assert lib.qlinear_codebook_workspace_bytes(5, 128, 128) == 0
+
+
+@pytest.mark.parametrize("fmt", [2, 4, 8])
+def test_grouped_params_layout(ql, fmt):
+    K, N = 384, 208          # 13 tiles: a full block and a ragged one; 3 units along K
+    G = K // 128
+    ntiles, nb = N // 16, (N // 16 + 7) // 8
+    def chunk(b, g, jj):
+        tb = min(8, ntiles - 8 * b)
+        return b * G * 8 + g * tb + jj
+    for group, ns in ((32, 4), (64, 2), (K, 1)):
+        rows = 1 if group == K else K // group
+        a = (np.arange(rows * N) % 2039).astype(np.float16).reshape(rows, N)
+        p = ql.qlinear_pack_params_grouped(fmt, group, a, N, K)
+        assert p.nbytes == ql.qlinear_params_bytes_grouped(fmt, group, N, K) == G * ns * N * 2
+        for (b, g, jj, ss, gi, h) in [(0, 0, 0, 0, 0, 0), (1, 2, 4, ns - 1, 7, 1), (0, 1, 3, ns // 2, 5, 0)]:
+            n = (8 * b + jj) * 16 + gi + 8 * h
+            src = 0 if group == K else g * ns + ss
+            assert p[(chunk(b, g, jj) * ns + ss) * 16 + gi * 2 + h] == a[src, n]
+    # group 128 matches the ungrouped packer
+    a = (np.arange(G * N) % 997).astype(np.float16).reshape(G, N)
+    assert np.array_equal(ql.qlinear_pack_params_grouped(fmt, 128, a, N, K),
+                          ql.qlinear_pack_params(fmt, a, N, K).reshape(-1))
+    lib = ql._lib
+    assert ql.qlinear_params_bytes_grouped(fmt, 96, N, K) == 0
+    assert ql.qlinear_params_bytes_grouped(16, 64, N, K) == 0
+    buf = np.zeros(64, dtype=np.uint16)
+    assert lib.qlinear_pack_params_grouped(16, 64, buf.ctypes.data, buf.ctypes.data, N, K) == 4
+    assert lib.qlinear_pack_params_grouped(fmt, 96, buf.ctypes.data, buf.ctypes.data, N, K) == 2
+    assert lib.qlinear_pack_params_grouped(fmt, 64, None, buf.ctypes.data, N, K) == 1

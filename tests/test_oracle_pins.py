@@ -278,3 +278,26 @@ def test_tilecoo_structure_and_bound():
     ebound.reshape(-1)[lay.positions] = np.abs(wf.reshape(-1)[lay.positions]) * 2.0 ** -11
     bound = np.abs(x.astype(np.float64)) @ ebound
     assert np.all(np.abs(y - x.astype(np.float64) @ wf) <= bound * (1 + 1e-9) + 1e-12)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("group", [32, 64, "K"])
+def test_finer_and_per_channel_groups_within_bound(bits, group):
+    """Groups of 32 and 64 and per-channel (one group of K): the element-wise min-max bound
+    and the layer bound hold with the group's own scales, so a group index taken at the
+    wrong granularity (for example k // 128) fails."""
+    K, N, M = 256, 24, 3
+    g = K if group == "K" else group
+    layer = gen.uniform_layer(81 + bits, K, N, bits, group=g)
+    assert layer.scales.shape == (K // g, N)
+    w = gen.weights(81 + bits, K, N).astype(np.float64)
+    deq = oracle.dequant_uniform(oracle.unpack_uniform(layer.qweight, bits), layer.scales,
+                                 layer.zeros, g)
+    el = _bound_uniform(layer, w)
+    assert np.all(np.abs(deq - w) <= el * (1 + 1e-12))
+    x = gen.activations(81, M, K)
+    y = oracle.gemv_uniform(x, layer.qweight, layer.scales, layer.zeros, bits, g)
+    bound = np.abs(x.astype(np.float64)) @ el
+    assert np.all(np.abs(y - x.astype(np.float64) @ w) <= bound * (1 + 1e-9) + 1e-12)
+    if g < 128:  # the finer scales really differ inside a 128-element span
+        assert not np.array_equal(layer.scales[0], layer.scales[1])

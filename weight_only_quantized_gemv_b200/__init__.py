@@ -58,6 +58,8 @@ _SIGS = {
     "qlinear_params_bytes": (_SZ, [_I, _I, _I]),
     "qlinear_pack": (_I, [_I, _P, _P, _I, _I]),
     "qlinear_pack_params": (_I, [_I, _P, _P, _I, _I]),
+    "qlinear_params_bytes_grouped": (_SZ, [_I, _I, _I, _I]),
+    "qlinear_pack_params_grouped": (_I, [_I, _I, _P, _P, _I, _I]),
     "qlinear_pack_tilecoo": (_I, [_P, _P, _P, _I, _I, _P, _P, _P]),
     "qlinear_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "qlinear_w4a16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
@@ -149,6 +151,26 @@ def qlinear_pack_params(fmt: int, canonical: np.ndarray, N: int, K: int) -> np.n
         raise QLinearError(2, "qlinear_pack_params")
     _check(_lib.qlinear_pack_params(fmt, _np_ptr(canonical), _np_ptr(out), N, K),
            "qlinear_pack_params")
+    return out
+
+
+def qlinear_params_bytes_grouped(fmt: int, group: int, N: int, K: int) -> int:
+    return int(_lib.qlinear_params_bytes_grouped(fmt, group, N, K))
+
+
+def qlinear_pack_params_grouped(fmt: int, group: int, canonical: np.ndarray, N: int,
+                                K: int) -> np.ndarray:
+    """fp16 [K / group, N] (or [1, N] for group = K) -> the kernel layout for that group."""
+    canonical = np.ascontiguousarray(canonical, dtype=np.float16)
+    rows = 1 if group == K else K // group
+    if canonical.shape != (rows, N):
+        raise QLinearError(2, "qlinear_pack_params_grouped")
+    nbytes = qlinear_params_bytes_grouped(fmt, group, N, K)
+    if nbytes == 0:
+        raise QLinearError(2, "qlinear_pack_params_grouped")
+    out = np.empty(nbytes // 2, dtype=np.float16)
+    _check(_lib.qlinear_pack_params_grouped(fmt, group, _np_ptr(canonical), _np_ptr(out), N, K),
+           "qlinear_pack_params_grouped")
     return out
 
 

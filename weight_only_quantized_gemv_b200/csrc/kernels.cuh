@@ -112,9 +112,15 @@ __host__ __device__ constexpr int default_wpu(int fmt, int mt) { return (mt == 1
 // taking tiles (8 / WPU) h .. (8 / WPU) (h + 1) - 1.  M1: exactly one row of x (only the
 // accumulator entries of batch column 0 are kept; x arrives by a 1-D bulk copy).  Every
 // other instance serves M >= 2 and copies x as one 2-D tile per unit through a tensor map.
-template <int FMT, int MT, bool OUTL, int WPU_, bool M1_ = false, int OCC_ = 0>
+template <int FMT, int MT, bool OUTL, int WPU_, bool M1_ = false, int OCC_ = 0, int NS_ = 1>
 struct Cfg {
   static constexpr bool M1 = M1_;
+  // quantization sub-groups per 128-k unit (group size 128 / NS): W2 / W4 / W8 only.  Each
+  // sub-group covers 8 / NS consecutive tensor-core steps (steps 2p, 2p + 1 hold k
+  // 32 p .. 32 p + 31), so its scale and zero pairs stay in registers for those steps.
+  static constexpr int NS = NS_;
+  static_assert(NS == 1 || NS == 2 || NS == 4, "group 128, 64 or 32");
+  static_assert(NS == 1 || (FMT != kLUT4 && !OUTL && WPU_ == 2), "finer groups: plain uniform formats, 2 warps per unit");
   static_assert(!M1 || MT == 1, "one row of x is the M <= 8 bucket");
   static constexpr int NC = 4;                       // consumer warps
   static constexpr int WPU = WPU_;
@@ -122,7 +128,7 @@ struct Cfg {
   static constexpr int NP = NC / WPU;                // warp groups, each takes whole units
   static constexpr int kTW = kBlockTiles / WPU;      // tiles of a unit per warp
   // tiles a warp holds in registers at once (independent accumulator chains)
-  static constexpr int kQ = kTW < 4 ? kTW : (MT == 2 || FMT == kW8) ? 2 : 4;
+  static constexpr int kQ = kTW < 4 ? kTW : (MT == 2 || FMT == kW8 || NS > 1) ? 2 : 4;
   static constexpr int T = 2;                        // tiles per warp in the block epilogue
   static constexpr int kThreads = (NC + 1) * 32;     // + one producer warp
   static constexpr int KW = Fmt<FMT>::kWords;
@@ -136,8 +142,9 @@ struct Cfg {
   static constexpr int kMinCtas = OCC_ ? OCC_ : (FMT == kLUT4) ? 2 : (MT == 1 && FMT != kW8) ? 3 : 2;
   static constexpr int kChunkBytes = 128 * KW;
   static constexpr int kCodeBytes = kBlockTiles * kChunkBytes;
-  static constexpr int kParamChunk = (FMT == kLUT4) ? 128 : 32;   // per tile, per array
-  static constexpr int kParamBytes = (FMT == kLUT4) ? 8 * 128 : 2 * 8 * 32;
+  static constexpr int kParamChunk = (FMT == kLUT4) ? 128 : 32 * NS;   // per tile, per array
+  static constexpr int kParamBytes = (FMT == kLUT4) ? 8 * 128 : 2 * 8 * 32 * NS;
+  static constexpr int kZeroOff = 8 * 32 * NS;   // zeros after the 8 tiles' scales
   // x rows in a stage: the 2-D tile copy (M >= 2) writes them densely; the single-row
   // kernel keeps 16 bytes of padding, which spreads the fragment loads over the banks
   static constexpr int kXStride = M1 ? 272 : 256;
@@ -354,9 +361,10 @@ __host__ __device__ __forceinline__ int cta_of_unit(int u, int U, int C) {
 
 // ---------------------------------------------------------------------------
 
-template <int FMT, int MT, bool OUTL, int WPU_, bool M1_ = false, int OCC_ = 0>
+template <int FMT, int MT, bool OUTL, int WPU_, bool M1_ = false, int OCC_ = 0, int NS_ = 1>
 struct Gemv {
-  using C_ = Cfg<FMT, MT, OUTL, WPU_, M1_, OCC_>;
+  using C_ = Cfg<FMT, MT, OUTL, WPU_, M1_, OCC_, NS_>;
+  static constexpr int NS = C_::NS;
   static constexpr int NC = C_::NC, T = C_::T, KW = C_::KW, NACC = C_::NACC, S = C_::S;
   static constexpr int WPU = C_::WPU, NP = C_::NP, kTW = C_::kTW;
   static constexpr bool kLut = (FMT == kLUT4);
@@ -666,8 +674,8 @@ struct Gemv {
         bulk_g2s(st + C_::kCodeBytes, static_cast<const float*>(P.zp) + ch * 32, param_bytes, full,
                  pol);
       } else {
-        bulk_g2s(st + C_::kCodeBytes, P.sc + ch * 16, param_bytes, full, pol);
-        bulk_g2s(st + C_::kCodeBytes + 256, static_cast<const __half*>(P.zp) + ch * 16,
+        bulk_g2s(st + C_::kCodeBytes, P.sc + ch * 16 * NS, param_bytes, full, pol);
+        bulk_g2s(st + C_::kCodeBytes + C_::kZeroOff, static_cast<const __half*>(P.zp) + ch * 16 * NS,
                  param_bytes, full, pol);
       }
     };
@@ -723,6 +731,10 @@ struct Gemv {
   __device__ static void unit(const GemvParams& P, uint8_t* smem, int i, int b, int warp,
                               int lane, float (&acc)[kTW][NACC], uint32_t (&orc)[3],
                               uint32_t (&oval)[3], int n) {
+    if constexpr (NS > 1) {
+      unit_fine(P, smem, i, b, warp, lane, acc);
+      return;
+    }
     const uint32_t ring = smem_addr(smem);
     const uint32_t bars = ring + C_::kBarOff;
     const uint32_t lut = ring + C_::kLutOff;
@@ -813,6 +825,146 @@ struct Gemv {
     }
   }
 
+  // One unit with NS quantization sub-groups (group 64 or 32; W2 / W4 / W8, two warps per
+  // unit, two quads of two tiles per warp).  Same stage protocol as unit(); per sub-group:
+  // its own sum of x and its own epilogue acc += s (d - z sum x), with that sub-group's
+  // scale and zero pairs held in registers (loaded with the codes).
+  struct QuadFine {
+    uint32_t w[kQ][KW];
+    uint32_t p0[kQ][NS], p1[kQ][NS];
+  };
+  __device__ static void load_quad_fine(uint32_t st, int j0, int lane, QuadFine& r) {
+    const int gi = lane >> 2;
+#pragma unroll
+    for (int i = 0; i < kQ; ++i) {
+      const uint32_t cb = st + (j0 + i) * C_::kChunkBytes + lane * 16;
+#pragma unroll
+      for (int q = 0; q < KW / 4; ++q) {
+        const uint4 v = lds128(cb + q * 512);
+        r.w[i][4 * q + 0] = v.x;
+        r.w[i][4 * q + 1] = v.y;
+        r.w[i][4 * q + 2] = v.z;
+        r.w[i][4 * q + 3] = v.w;
+      }
+#pragma unroll
+      for (int ss = 0; ss < NS; ++ss) {
+        const uint32_t po = ((j0 + i) * NS + ss) * 32 + gi * 4;
+        r.p0[i][ss] = lds32(st + C_::kCodeBytes + po);
+        r.p1[i][ss] = lds32(st + C_::kCodeBytes + C_::kZeroOff + po);
+      }
+    }
+  }
+  __device__ static void compute_quad_fine(const QuadFine& r, const uint4 (&xr)[4],
+                                           const uint4 (&xr2)[4], const float (&cx)[NS][NACC],
+                                           float (*acc)[NACC]) {
+    constexpr int kSub = 8 / NS;  // steps per sub-group
+    const auto& w = r.w;
+#pragma unroll
+    for (int ss = 0; ss < NS; ++ss) {
+      float c[kQ][NACC];
+      float co[(FMT == kW2) ? kQ : 1][NACC];
+#pragma unroll
+      for (int s = ss * kSub; s < (ss + 1) * kSub; ++s) {
+        const int p = s >> 1, h = s & 1;
+        const uint32_t b0 = h ? xr[p].z : xr[p].x, b1 = h ? xr[p].w : xr[p].y;
+        uint32_t b2 = 0, b3 = 0;
+        if constexpr (MT == 2) {
+          b2 = h ? xr2[p].z : xr2[p].x;
+          b3 = h ? xr2[p].w : xr2[p].y;
+        }
+#pragma unroll
+        for (int i = 0; i < kQ; ++i) {
+          uint32_t a[4];
+          frag_uniform<FMT>(w[i], s, a);
+          if constexpr (FMT == kW2) {
+            if (h == 1) {  // odd steps accumulate separately (their codes carry x16)
+              if (s == ss * kSub + 1) {
+                hmma0(&co[i][0], a, b0, b1);
+                if constexpr (MT == 2) hmma0(&co[i][4], a, b2, b3);
+              } else {
+                hmma(&co[i][0], a, b0, b1);
+                if constexpr (MT == 2) hmma(&co[i][4], a, b2, b3);
+              }
+              continue;
+            }
+          }
+          if (s == ss * kSub) {
+            hmma0(&c[i][0], a, b0, b1);
+            if constexpr (MT == 2) hmma0(&c[i][4], a, b2, b3);
+          } else {
+            hmma(&c[i][0], a, b0, b1);
+            if constexpr (MT == 2) hmma(&c[i][4], a, b2, b3);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kQ; ++i) {
+        const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&r.p0[i][ss]));
+        const float2 z2 = __half22float2(*reinterpret_cast<const __half2*>(&r.p1[i][ss]));
+#pragma unroll
+        for (int e = 0; e < NACC; ++e) {
+          if (C_::M1 && (e & 1)) continue;  // batch column 1 of the fragment: no such row
+          float d = c[i][e];
+          if constexpr (FMT == kW2) d = fmaf(co[i][e], 0.0625f, d);  // odd steps carry x16
+          const float sc = (e & 2) ? s2.y : s2.x;
+          const float zc = (e & 2) ? z2.y : z2.x;
+          acc[i][e] = fmaf(sc, fmaf(-zc, cx[ss][e], d), acc[i][e]);
+        }
+      }
+    }
+  }
+  __device__ static void unit_fine(const GemvParams& P, uint8_t* smem, int i, int b, int warp,
+                                   int lane, float (&acc)[kTW][NACC]) {
+    static_assert(kTW == 2 * kQ, "two quads per warp");
+    constexpr int kSub = 8 / NS;
+    const uint32_t ring = smem_addr(smem);
+    const uint32_t bars = ring + C_::kBarOff;
+    const int sub = warp % WPU;
+    const int s = i % S;
+    const int tb = tiles_in_block(b, P.ntiles);
+    const uint32_t st = ring + s * C_::kStageBytes;
+    if (!mbar_wait(bars + 8 * s, (i / S) & 1)) atomicOr(P.err, kErrFullTimeout);
+    uint4 xr[4], xr2[4];
+    read_x(P, st, lane, xr, xr2);
+    const int t0 = kTW * sub;
+    const int nq = tb <= t0 ? 0 : (tb - t0 >= kTW ? kTW / kQ : (tb - t0 + kQ - 1) / kQ);
+    const uint32_t empty = bars + 8 * (S + s);
+    // sums of x over each sub-group, in the row scales of the codes
+    float cx[NS][NACC];
+    {
+      const uint32_t ones[4] = {kOnesLo, Fmt<FMT>::kOnesHi, kOnesLo, Fmt<FMT>::kOnesHi};
+#pragma unroll
+      for (int s8 = 0; s8 < 8; ++s8) {
+        const int p = s8 >> 1, h = s8 & 1, ss = s8 / kSub;
+        if (s8 % kSub == 0) {
+          hmma0(&cx[ss][0], ones, h ? xr[p].z : xr[p].x, h ? xr[p].w : xr[p].y);
+          if constexpr (MT == 2)
+            hmma0(&cx[ss][4], ones, h ? xr2[p].z : xr2[p].x, h ? xr2[p].w : xr2[p].y);
+        } else {
+          hmma(&cx[ss][0], ones, h ? xr[p].z : xr[p].x, h ? xr[p].w : xr[p].y);
+          if constexpr (MT == 2)
+            hmma(&cx[ss][4], ones, h ? xr2[p].z : xr2[p].x, h ? xr2[p].w : xr2[p].y);
+        }
+      }
+    }
+    {
+      QuadFine q0;
+      load_quad_fine(st, t0, lane, q0);
+      if (nq <= 1) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty);
+      }
+      if (nq >= 1) compute_quad_fine(q0, xr, xr2, cx, acc);
+    }
+    if (nq > 1) {
+      QuadFine q1;
+      load_quad_fine(st, t0 + kQ, lane, q1);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty);
+      compute_quad_fine(q1, xr, xr2, cx, acc + kQ);
+    }
+  }
+
   // Entries of unit i a thread takes first (index `slot` of the WPU x 32 threads of the
   // group, then every WPU x 32-th), held in registers one unit ahead.
   static constexpr int kOutPre = 3 - (WPU > 1) - (WPU > 2);
@@ -869,14 +1021,14 @@ struct NoXMap {
 template <bool XT> struct XMapParam { using type = NoXMap; };
 template <> struct XMapParam<true> { using type = CUtensorMap; };
 
-template <int FMT, int MT, bool OUTL, int WPU, bool M1, int OCC>
-__global__ void __launch_bounds__(Cfg<FMT, MT, OUTL, WPU, M1, OCC>::kThreads,
-                                  Cfg<FMT, MT, OUTL, WPU, M1, OCC>::kMinCtas)
+template <int FMT, int MT, bool OUTL, int WPU, bool M1, int OCC, int NS = 1>
+__global__ void __launch_bounds__(Cfg<FMT, MT, OUTL, WPU, M1, OCC, NS>::kThreads,
+                                  Cfg<FMT, MT, OUTL, WPU, M1, OCC, NS>::kMinCtas)
     qgemv_kernel(const GemvParams P, const __grid_constant__ typename XMapParam<!M1>::type xm) {
   const CUtensorMap* xmap = nullptr;
   if constexpr (!M1) xmap = &xm;
-  using G_ = Gemv<FMT, MT, OUTL, WPU, M1, OCC>;
-  using C_ = Cfg<FMT, MT, OUTL, WPU, M1, OCC>;
+  using G_ = Gemv<FMT, MT, OUTL, WPU, M1, OCC, NS>;
+  using C_ = Cfg<FMT, MT, OUTL, WPU, M1, OCC, NS>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int u0 = unit_begin(blockIdx.x, P.U, P.C);

@@ -141,3 +141,48 @@ extern "C" ql_status qlinear_pack_tilecoo(const uint32_t* offsets, const uint8_t
     }
   return QL_OK;
 }
+
+// Sub-groups per 128-k unit for a group size: 4 (g = 32), 2 (64), 1 (128, or per-channel
+// g = K, whose one parameter per column is repeated in every 128-k unit); 0 if unsupported.
+static int subgroups(int group, int K) {
+  if (group == 32) return 4;
+  if (group == 64) return 2;
+  if (group == kGroup || group == K) return 1;
+  return 0;
+}
+
+extern "C" size_t qlinear_params_bytes_grouped(int fmt, int group, int N, int K) {
+  if (fmt != kW2 && fmt != kW4 && fmt != kW8) return 0;
+  if (!shape_ok(N, K) || !subgroups(group, K)) return 0;
+  return (size_t)(K / kGroup) * subgroups(group, K) * N * sizeof(uint16_t);
+}
+
+extern "C" ql_status qlinear_pack_params_grouped(int fmt, int group, const void* canonical,
+                                                 void* packed, int N, int K) {
+  if (fmt != kW2 && fmt != kW4 && fmt != kW8) return QL_ERR_UNSUPPORTED;
+  if (!canonical || !packed) return QL_ERR_NULL;
+  const int NS = subgroups(group, K);
+  if (!shape_ok(N, K) || !NS) return QL_ERR_SHAPE;
+  const bool per_channel = group == K && group != kGroup;
+  const int G = K / kGroup;
+  const int ntiles = N / kTileN;
+  const int nblocks = (ntiles + kBlockTiles - 1) / kBlockTiles;
+  const uint16_t* a = static_cast<const uint16_t*>(canonical);
+  uint16_t* o = static_cast<uint16_t*>(packed);
+  for (int b = 0; b < nblocks; ++b) {
+    const int tb = tiles_in_block(b, ntiles);
+    for (int g = 0; g < G; ++g)
+      for (int jj = 0; jj < tb; ++jj) {
+        const long long c = chunk_index(b, g, jj, G, ntiles);
+        const int n_base = (b * kBlockTiles + jj) * kTileN;
+        for (int ss = 0; ss < NS; ++ss)
+          for (int gi = 0; gi < 8; ++gi)
+            for (int h = 0; h < 2; ++h) {
+              const int n = n_base + gi + 8 * h;
+              const int src_group = per_channel ? 0 : g * NS + ss;
+              o[(c * NS + ss) * 16 + gi * 2 + h] = a[(size_t)src_group * N + n];
+            }
+      }
+  }
+  return QL_OK;
+}

@@ -30,6 +30,7 @@ struct Plan {
   int nblocks, ntiles, G, MT, WPU, NC, T, threads, smem;
   bool M1;          // W4 with one row of x: the kernel keeps only batch column 0
   bool OCC2;        // ... with registers for two CTAs per SM (grids of at most 2 per SM)
+  int NS;           // quantization sub-groups per 128-k unit (group 128 / NS)
   size_t counter_offset, partial_offset, ws_bytes;
 };
 
@@ -40,11 +41,33 @@ struct KernelInfo {
 };
 
 template <int FMT, int MT, bool OUTL, int WPU = qlk::default_wpu(FMT, MT), bool M1 = false,
-          int OCC = 0>
+          int OCC = 0, int NS = 1>
 KernelInfo kernel_info() {
-  using C = qlk::Cfg<FMT, MT, OUTL, WPU, M1, OCC>;
-  return KernelInfo{reinterpret_cast<const void*>(qlk::qgemv_kernel<FMT, MT, OUTL, WPU, M1, OCC>),
-                    C::kThreads, C::kSmemBytes, C::NC, C::T, !M1};
+  using C = qlk::Cfg<FMT, MT, OUTL, WPU, M1, OCC, NS>;
+  return KernelInfo{
+      reinterpret_cast<const void*>(qlk::qgemv_kernel<FMT, MT, OUTL, WPU, M1, OCC, NS>),
+      C::kThreads, C::kSmemBytes, C::NC, C::T, !M1};
+}
+
+// Finer quantization groups (NS sub-groups per 128-k unit): two warps per unit for every
+// format, so each warp holds two quads of two tiles (the sub-groups' scale and zero pairs
+// take registers that four tiles at a time would not leave).
+constexpr int kFineWpu = 2;
+
+template <int FMT, int NS>
+KernelInfo fine_kernel(int MT, bool m1) {
+  if (MT == 2) return kernel_info<FMT, 2, false, kFineWpu, false, 0, NS>();
+  return m1 ? kernel_info<FMT, 1, false, kFineWpu, true, 0, NS>()
+            : kernel_info<FMT, 1, false, kFineWpu, false, 0, NS>();
+}
+
+template <int NS>
+KernelInfo fine_kernel_fmt(int fmt, int MT, bool m1) {
+  switch (fmt) {
+    case kW2: return fine_kernel<kW2, NS>(MT, m1);
+    case kW8: return fine_kernel<kW8, NS>(MT, m1);
+    default: return fine_kernel<kW4, NS>(MT, m1);
+  }
 }
 
 // The M <= 8 kernel of a format: its single-row variant for M = 1, else the one for M >= 2.
@@ -62,7 +85,10 @@ KernelInfo w4_m8_kernel(bool m1) {
   return m1 ? kernel_info<kW4, 1, false, WPU, true>() : kernel_info<kW4, 1, false, WPU, false>();
 }
 
-KernelInfo select_kernel(int fmt, int MT, bool outl, int wpu, bool m1, bool occ2 = false) {
+KernelInfo select_kernel(int fmt, int MT, bool outl, int wpu, bool m1, bool occ2 = false,
+                         int ns = 1) {
+  if (ns == 2) return fine_kernel_fmt<2>(fmt, MT, m1);
+  if (ns == 4) return fine_kernel_fmt<4>(fmt, MT, m1);
   if (occ2 && fmt == kW4 && MT == 1 && !outl && wpu == 1 && m1)
     return kernel_info<kW4, 1, false, 1, true, 2>();
   if (outl) return MT == 1 ? m8_kernel<kW4, true>(m1) : kernel_info<kW4, 2, true>();
@@ -100,7 +126,7 @@ cudaError_t prepare_kernel(const KernelInfo& k, int dev, int* ctas) {
   return cudaSuccess;
 }
 
-cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
+cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p, int ns = 1) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -108,10 +134,11 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   p->MT = M <= 8 ? 1 : 2;
-  p->WPU = qlk::default_wpu(fmt, p->MT);
+  p->WPU = ns > 1 ? kFineWpu : qlk::default_wpu(fmt, p->MT);
   p->M1 = M == 1;
   p->OCC2 = false;
-  const KernelInfo k = select_kernel(fmt, p->MT, outl, p->WPU, p->M1);
+  p->NS = ns;
+  const KernelInfo k = select_kernel(fmt, p->MT, outl, p->WPU, p->M1, false, ns);
   int occ = 1;
   e = prepare_kernel(k, dev, &occ);
   if (e != cudaSuccess) return e;
@@ -144,7 +171,7 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
   //    block that fit instead: C = nblocks * k is still block-aligned, because CTA c covers
   //    units [c G / k, (c + 1) G / k) of block c / k.
   bool small_m1 = false;
-  if (p->M1 && fmt == kW4 && !outl) {
+  if (p->M1 && fmt == kW4 && !outl && ns == 1) {
     const long long c2 = 2LL * sms, kmax = c2 / p->nblocks;
     if (kmax >= 1 && p->U <= 16 * p->nblocks * kmax) {
       long long kd = kmax;
@@ -174,7 +201,7 @@ cudaError_t make_plan(int fmt, int M, int N, int K, bool outl, Plan* p) {
   // shortens the one unit a warp would otherwise work through alone.  The M = 1 kernel
   // (half the epilogue) is fastest with one warp per unit on every layer measured.
   // QLINEAR_WPU = 1, 2 or 4 overrides.
-  if (fmt == kW4 && p->MT == 1 && !outl) {
+  if (fmt == kW4 && p->MT == 1 && !outl && ns == 1) {
     const long long per_cta = (p->U + C - 1) / C;
     int wpu = p->M1 ? 1 : per_cta <= 4 ? 4 : per_cta <= 24 ? 2 : 1;
     if (pol.wpu > 0) wpu = pol.wpu;
@@ -264,7 +291,17 @@ struct Call {
   void* ws;
   size_t ws_bytes;
   cudaStream_t stream;
+  int ns = 1;  // sub-groups per 128-k unit (from the group size)
 };
+
+// sub-groups per 128-k unit for a group size of the uniform formats: 4 (32), 2 (64),
+// 1 (128, or per-channel g = K with the parameters repeated per unit by the packer)
+int subgroups(int group, int K) {
+  if (group == 32) return 4;
+  if (group == 64) return 2;
+  if (group == kGroup || group == K) return 1;
+  return 0;
+}
 
 ql_status run(const Call& c) {
   if (!c.x || !c.qw || !c.p0 || !c.p1 || !c.y) return QL_ERR_NULL;
@@ -281,7 +318,7 @@ ql_status run(const Call& c) {
   if (c.outl && (!aligned(c.toff, 4) || !aligned(c.trc, 2) || !aligned(c.tval, 2)))
     return QL_ERR_ALIGN;
   Plan p;
-  if (make_plan(c.fmt, c.M, c.N, c.K, c.outl, &p) != cudaSuccess) return QL_ERR_CUDA;
+  if (make_plan(c.fmt, c.M, c.N, c.K, c.outl, &p, c.ns) != cudaSuccess) return QL_ERR_CUDA;
   if (!c.ws || c.ws_bytes < p.ws_bytes) return QL_ERR_WORKSPACE;
   if (!aligned(c.ws, 16)) return QL_ERR_ALIGN;
   qlk::GemvParams P;
@@ -304,7 +341,7 @@ ql_status run(const Call& c) {
   P.ntiles = p.ntiles;
   P.U = (int)p.U;
   P.C = p.C;
-  const KernelInfo k = select_kernel(c.fmt, p.MT, c.outl, p.WPU, p.M1, p.OCC2);
+  const KernelInfo k = select_kernel(c.fmt, p.MT, c.outl, p.WPU, p.M1, p.OCC2, p.NS);
   // Programmatic stream serialization: the kernel may start while the previous kernel in
   // the stream drains; it requests only static weight bytes before griddepcontrol.wait.
   cudaLaunchConfig_t cfg = {};
@@ -451,6 +488,14 @@ extern "C" size_t qlinear_workspace_bytes(int fmt, int M, int N, int K) {
   if (!fmt_ok(fmt) || !shape_ok(M, N, K)) return 0;
   Plan p;
   if (make_plan(fmt, M, N, K, false, &p) != cudaSuccess) return 0;
+  // the finer-group kernels (group 64, 32) may resolve to another occupancy: cover them
+  if (fmt != kLUT4) {
+    for (int ns : {2, 4}) {
+      Plan q;
+      if (make_plan(fmt, M, N, K, false, &q, ns) == cudaSuccess && q.ws_bytes > p.ws_bytes)
+        p.ws_bytes = q.ws_bytes;
+    }
+  }
   // the outlier kernel (W4) may resolve to a different occupancy: cover both
   if (fmt == kW4 && N % 128 == 0) {
     Plan q;
@@ -478,9 +523,10 @@ extern "C" ql_status qlinear_plan(int fmt, int M, int N, int K, ql_plan* plan) {
   extern "C" ql_status NAME(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,  \
                             const uint16_t* zeros, uint16_t* y, int M, int N, int K, int group,  \
                             void* workspace, size_t workspace_bytes, ql_stream_t stream) {       \
-    if (group != kGroup) return QL_ERR_SHAPE;                                                     \
+    const int ns = subgroups(group, K);                                                           \
+    if (!ns) return QL_ERR_SHAPE;                                                                 \
     Call c{FMT, false, x, qweight, scales, zeros, nullptr, nullptr, nullptr, y, M, N, K,         \
-           workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)};                   \
+           workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), ns};               \
     return run(c);                                                                                \
   }
 

@@ -15,7 +15,8 @@ import torch
 from . import (QL_FMT_LUT4, QL_FMT_W2, QL_FMT_W4, QL_FMT_W8, QL_STRATEGY_PREFILL,
                qlinear_debug_dequant, qlinear_policy_lookup,
                qlinear_debug_unpack, qlinear_dequant_fp16, qlinear_lut4, qlinear_pack,
-               qlinear_matmul, qlinear_pack_params, qlinear_prefill,
+               qlinear_matmul, qlinear_pack_params, qlinear_pack_params_grouped,
+               qlinear_prefill,
                qlinear_pack_tilecoo, qlinear_w2a16, qlinear_w4a16, qlinear_w4a16_outlier,
                qlinear_w8a16, qlinear_workspace_bytes)
 
@@ -31,8 +32,9 @@ class QuantLinear:
 
     def __init__(self, fmt: int, K: int, N: int, canonical_codes: np.ndarray,
                  p0: np.ndarray, p1: Optional[np.ndarray] = None,
-                 tilecoo: Optional[tuple] = None, device="cuda", max_m: int = 16):
-        self.fmt, self.K, self.N = fmt, K, N
+                 tilecoo: Optional[tuple] = None, device="cuda", max_m: int = 16,
+                 group: int = 128):
+        self.fmt, self.K, self.N, self.group = fmt, K, N, group
         self.device = torch.device(device)
         packed = qlinear_pack(fmt, canonical_codes, N, K)
         self.qweight = _dev(packed, self.device)
@@ -40,6 +42,11 @@ class QuantLinear:
             self.p0 = _dev(np.asarray(p0, dtype=np.float16).view(np.uint16), self.device)  # lut16
             self.p1 = _dev(qlinear_pack_params(fmt, np.asarray(p1, dtype=np.float32), N, K),
                            self.device)  # absmax
+        elif group != 128:
+            self.p0 = _dev(qlinear_pack_params_grouped(fmt, group, p0, N, K).view(np.uint16),
+                           self.device)  # scales, one per (sub-group, column)
+            self.p1 = _dev(qlinear_pack_params_grouped(fmt, group, p1, N, K).view(np.uint16),
+                           self.device)  # zeros
         else:
             self.p0 = _dev(qlinear_pack_params(fmt, np.asarray(p0, dtype=np.float16), N, K)
                            .view(np.uint16), self.device)  # scales
@@ -76,11 +83,16 @@ class QuantLinear:
                          self.workspace, stream)
         else:
             _ENTRY[self.fmt](xv, self.qweight, self.p0, self.p1, yv, M, self.N, self.K,
-                             self.workspace, stream)
+                             self.workspace, stream, group=self.group)
         return y
+
+    def _group128(self, what: str) -> None:
+        if self.group != 128:
+            raise ValueError(f"{what} reads parameters packed for group 128")
 
     def dequant_fp16(self, w: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
         """The dense fp16 weights, ``w[N, K]`` (one row per output column)."""
+        self._group128("dequant_fp16")
         if w is None:
             w = torch.empty((self.N, self.K), dtype=torch.float16, device=self.device)
         qlinear_dequant_fp16(self.fmt, self.qweight, self.p0, self.p1, w.view(torch.int16),
@@ -93,6 +105,7 @@ class QuantLinear:
         by the layer when not given), then one dense GEMM.  Dense part only (no outliers)."""
         if self.tile is not None:
             raise ValueError("prefill covers the dense formats; the outlier layer has none")
+        self._group128("prefill")
         M = x.shape[0]
         if y is None:
             y = torch.empty((M, self.N), dtype=torch.float16, device=self.device)
@@ -112,6 +125,7 @@ class QuantLinear:
         buffer for prefill is allocated on the first call the policy sends to prefill."""
         if self.tile is not None:
             raise ValueError("the policy map covers the dense formats")
+        self._group128("matmul")
         M = x.shape[0]
         if y is None:
             y = torch.empty((M, self.N), dtype=torch.float16, device=self.device)
@@ -132,15 +146,17 @@ class QuantLinear:
         return codes
 
     def debug_dequant(self, stream=None) -> torch.Tensor:
+        self._group128("debug_dequant")
         w = torch.empty((self.K, self.N), dtype=torch.float32, device=self.device)
         qlinear_debug_dequant(self.fmt, self.qweight, self.p0, self.p1, w, self.N, self.K, stream)
         return w
 
 
 def from_uniform(layer, device="cuda", max_m: int = 16) -> QuantLinear:
-    """From a ``synth.gen.UniformLayer``-like object (bits, K, N, qweight, scales, zeros)."""
+    """From a ``synth.gen.UniformLayer``-like object (bits, K, N, qweight, scales, zeros and,
+    optionally, group)."""
     return QuantLinear(layer.bits, layer.K, layer.N, layer.qweight, layer.scales, layer.zeros,
-                       device=device, max_m=max_m)
+                       device=device, max_m=max_m, group=getattr(layer, "group", 128))
 
 
 def from_lut4(layer, device="cuda", max_m: int = 16) -> QuantLinear:

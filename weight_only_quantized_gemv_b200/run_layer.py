@@ -24,12 +24,13 @@ from . import (FORMATS, QL_FMT_LUT4, qlinear_lut4, qlinear_plan, qlinear_read_er
 _UNIFORM = {2: qlinear_w2a16, 4: qlinear_w4a16, 8: qlinear_w8a16}
 
 
-def algorithmic_bytes(fmt: int, K: int, N: int, M: int, nnz: int = 0) -> int:
+def algorithmic_bytes(fmt: int, K: int, N: int, M: int, nnz: int = 0, group: int = 128) -> int:
     """Bytes a launch must move at least: codes, parameters, x and y (and the Tile-COO
-    arrays: 2-byte (row, col) and 2-byte value per outlier, 4-byte offset per tile)."""
+    arrays: 2-byte (row, col) and 2-byte value per outlier, 4-byte offset per tile).
+    Per-channel parameters (group = K) count once per column."""
     if fmt == QL_FMT_LUT4:
         return K * N // 2 + (K // 64) * N * 4 + 32 + M * K * 2 + M * N * 2
-    b = K * N * fmt // 8 + 2 * (K // 128) * N * 2 + M * K * 2 + M * N * 2
+    b = K * N * fmt // 8 + 2 * (K // group) * N * 2 + M * K * 2 + M * N * 2
     if nnz:
         b += 4 * nnz + 4 * ((K // 128) * (N // 128) + 1)
     return b
@@ -45,6 +46,8 @@ def main() -> None:
     ap.add_argument("--copies", type=int, default=3)
     ap.add_argument("--time", action="store_true")
     ap.add_argument("--outliers", type=float, default=0.0)
+    ap.add_argument("--group", type=int, default=128,
+                    help="W2/W4/W8 group size: 128, 64, 32, or K (per-channel)")
     a = ap.parse_args()
     fmt, K, N, M = FORMATS[a.fmt], a.K, a.N, a.M
     if a.outliers and (a.fmt != "w4" or N % 128):
@@ -60,9 +63,11 @@ def main() -> None:
         p0 = [torch.linspace(-1, 1, 16, device=dev).half().view(torch.int16)] * a.copies
         p1 = [torch.rand((K // 64) * N, device=dev, generator=gen) * 0.05 for _ in range(a.copies)]
     else:
-        p0 = [(torch.rand(G * N, device=dev, generator=gen) * 0.01).half().view(torch.int16)
+        # packed parameter entries: one per (sub-group, column); per-channel ones repeat per 128
+        PG = G * (128 // a.group if a.group < 128 else 1)
+        p0 = [(torch.rand(PG * N, device=dev, generator=gen) * 0.01).half().view(torch.int16)
               for _ in range(a.copies)]
-        p1 = [torch.randint(0, 1 << bits, (G * N,), device=dev, generator=gen).half().view(torch.int16)
+        p1 = [torch.randint(0, 1 << bits, (PG * N,), device=dev, generator=gen).half().view(torch.int16)
               for _ in range(a.copies)]
     x = torch.randn(M, K, device=dev, generator=gen).half().view(torch.int16)
     y = torch.empty(M, N, device=dev, dtype=torch.int16)
@@ -86,7 +91,7 @@ def main() -> None:
         elif fmt == QL_FMT_LUT4:
             qlinear_lut4(x, q[c], p0[c], p1[c], y, M, N, K, ws)
         else:
-            _UNIFORM[fmt](x, q[c], p0[c], p1[c], y, M, N, K, ws)
+            _UNIFORM[fmt](x, q[c], p0[c], p1[c], y, M, N, K, ws, group=a.group)
 
     if not a.time:
         for i in range(a.launches):
@@ -112,8 +117,10 @@ def main() -> None:
     e1.record()
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / (reps * a.launches)
-    b = algorithmic_bytes(fmt, K, N, M, nnz) + (4 * ((K // 128) * (N // 128) + 1) if outl and not nnz else 0)
-    print(json.dumps({"fmt": a.fmt, "K": K, "N": N, "M": M, "nnz": nnz, "us": round(us, 3), "bytes": b,
+    b = algorithmic_bytes(fmt, K, N, M, nnz, group=a.group) + \
+        (4 * ((K // 128) * (N // 128) + 1) if outl and not nnz else 0)
+    print(json.dumps({"fmt": a.fmt, "group": a.group, "K": K, "N": N, "M": M, "nnz": nnz,
+                      "us": round(us, 3), "bytes": b,
                       "GBs": round(b / us / 1e3, 1), "ctas": qlinear_plan(fmt, M, N, K).ctas,
                       "error_flags": qlinear_read_error(ws)}))
 
