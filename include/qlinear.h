@@ -3,6 +3,10 @@
  *
  *   y[M, N] = x[M, K] . dequant(Wq)[K, N],   M = 1..16 activation rows (LLM decoding)
  *
+ * Also: a prefill path for any M (stand-alone dequantization to fp16 + one dense GEMM), a
+ * measured policy map with a dispatcher for any M, and a codebook GEMV with a Psumbook
+ * (sections further down).
+ *
  * Formats
  *   W2 / W4 / W8 : group-wise asymmetric uniform codes, one fp16 scale s and one
  *                  fp16 zero z (an integer) per 128-element group along K per
