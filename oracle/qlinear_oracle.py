@@ -3,8 +3,10 @@
 Test infrastructure only (see the package docstring).  Every function reads
 the canonical layouts:
 
-* uniform b-bit codes: ``uint32[K / P, N]``, ``P = 32 / b``, word ``(j, n)``
-  bits ``[b*i, b*i + b)`` hold the code of weight ``(P*j + i, n)``;
+* uniform b-bit codes: ``uint32[K * b / 32, N]``, each column one little-endian
+  bit stream with code k in bits ``[b*k, b*k + b)`` (for b = 2, 4, 8: word
+  ``(j, n)`` bits ``[b*i, b*i + b)`` hold the code of weight ``(P*j + i, n)``,
+  ``P = 32 / b``; 3-bit codes straddle words, 32 codes per 3 words);
 * scales, zeros: fp16 ``[K / g, N]`` (zeros hold integers);
 * LUT4 codes: ``uint8[K / 2, N]``, low nibble = even k; ``absmax`` fp32
   ``[K / 64, N]``; ``lut`` fp16 ``[16]``;
@@ -60,14 +62,27 @@ def _col_select(a: np.ndarray, cols: Optional[Sequence[int]]) -> np.ndarray:
 
 
 def unpack_uniform(qweight: np.ndarray, bits: int, cols: Optional[Sequence[int]] = None) -> np.ndarray:
-    """Canonical ``uint32[K / P, N]`` words -> ``uint8[K, N]`` codes."""
+    """Canonical words -> ``uint8[K, N]`` codes.  Each column's words form one little-endian
+    bit stream (word j = stream bits 32 j .. 32 j + 31); code k is stream bits
+    ``[bits*k, bits*k + bits)``.  For bits dividing 32 this reads ``P = 32 / bits`` whole
+    codes per word; 3-bit codes may straddle two words."""
     words = _col_select(qweight, cols).astype(np.uint32)
-    P = 32 // bits
     mask = np.uint32((1 << bits) - 1)
-    KP, N = words.shape
-    codes = np.empty((KP * P, N), dtype=np.uint8)
-    for i in range(P):
-        codes[i::P, :] = (words >> np.uint32(bits * i)) & mask
+    W, N = words.shape
+    if 32 % bits == 0:
+        P = 32 // bits
+        codes = np.empty((W * P, N), dtype=np.uint8)
+        for i in range(P):
+            codes[i::P, :] = (words >> np.uint32(bits * i)) & mask
+        return codes
+    K = W * 32 // bits
+    w64 = words.astype(np.uint64)
+    nxt = np.vstack([w64[1:], np.zeros((1, N), dtype=np.uint64)])
+    pair = w64 | (nxt << np.uint64(32))        # stream bits 32 j .. 32 j + 63
+    codes = np.empty((K, N), dtype=np.uint8)
+    for k in range(K):
+        o = bits * k
+        codes[k] = (pair[o // 32] >> np.uint64(o % 32)) & np.uint64(mask)
     return codes
 
 

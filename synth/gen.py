@@ -15,9 +15,11 @@ What is produced, and the recipe each follows
   scale is ``s = fp16(s32)``, ``z = clip(rint(-min / s), 0, 2^b - 1)`` and
   ``q = clip(rint(w / s) + z, 0, 2^b - 1)``, the last two in fp64 with the
   stored fp16 ``s``.  A group whose stored scale is 0 stores s = z = q = 0.
-* Canonical code layout ``uint32[K / P, N]`` with ``P = 32 / b`` codes per
-  word packed along K: word ``(j, n)`` bits ``[b*i, b*i + b)`` hold
-  ``q[P*j + i, n]``.
+* Canonical code layout ``uint32[K * b / 32, N]``: each column's codes form one
+  little-endian bit stream along K, code k in bits ``[b*k, b*k + b)``, 32 bits per
+  word.  For b = 2, 4, 8 word ``(j, n)`` bits ``[b*i, b*i + b)`` hold
+  ``q[P*j + i, n]`` (``P = 32 / b``); 3-bit codes (b = 3, the GPTQ-style packing
+  of 32 codes in 3 words) run across word boundaries.
 * LUT4 (the NF4-style format of the "Fast NF4 Dequantization Kernels" page):
   a sorted 16-entry fp16 table holding -1, 0, +1 and 13 further distinct
   values drawn from U(-1, 1); an fp32 ``absmax`` per 64-element block along K
@@ -88,16 +90,30 @@ def activations(seed: int, M: int, K: int) -> np.ndarray:
 
 
 def pack_codes(codes: np.ndarray, bits: int) -> np.ndarray:
-    """``uint8[K, N]`` codes -> canonical ``uint32[K / P, N]``."""
+    """``uint8[K, N]`` codes -> canonical ``uint32[K * bits / 32, N]``: each column is one
+    little-endian bit stream, code k in bits ``[bits*k, bits*k + bits)``, 32 bits per word.
+    For bits dividing 32 that is ``P = 32 / bits`` whole codes per word; 3-bit codes run
+    across word boundaries (32 codes in 3 words)."""
     K, N = codes.shape
-    P = 32 // bits
-    if K % P:
-        raise ValueError("K must be a multiple of the codes per word")
-    c = codes.reshape(K // P, P, N).astype(np.uint32)
-    out = np.zeros((K // P, N), dtype=np.uint32)
-    for i in range(P):
-        out |= c[:, i, :] << np.uint32(bits * i)
-    return out
+    if (K * bits) % 32:
+        raise ValueError("K * bits must be a multiple of 32")
+    if 32 % bits == 0:
+        P = 32 // bits
+        c = codes.reshape(K // P, P, N).astype(np.uint32)
+        out = np.zeros((K // P, N), dtype=np.uint32)
+        for i in range(P):
+            out |= c[:, i, :] << np.uint32(bits * i)
+        return out
+    W = K * bits // 32
+    out = np.zeros((W + 1, N), dtype=np.uint64)     # one spare word for the last straddle
+    c = codes.astype(np.uint64)
+    for k in range(K):
+        o = bits * k
+        j, sh = o // 32, o % 32
+        out[j] |= (c[k] << np.uint64(sh)) & np.uint64(0xFFFFFFFF)
+        if sh + bits > 32:
+            out[j + 1] |= c[k] >> np.uint64(32 - sh)
+    return out[:W].astype(np.uint32)
 
 
 def pack_nibbles(codes: np.ndarray) -> np.ndarray:
@@ -119,7 +135,7 @@ class UniformLayer:
     N: int
     group: int
     codes: np.ndarray      # uint8[K, N] (kept for the generator's own checks)
-    qweight: np.ndarray    # uint32[K / P, N] canonical
+    qweight: np.ndarray    # uint32[K * bits / 32, N] canonical
     scales: np.ndarray     # fp16[K / group, N]
     zeros: np.ndarray      # fp16[K / group, N] (integers)
     scales32: np.ndarray   # fp32[K / group, N]: the pre-rounding fp32 scale
