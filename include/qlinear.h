@@ -8,7 +8,7 @@
  * (sections further down).
  *
  * Formats
- *   W2 / W4 / W8 : group-wise asymmetric uniform codes, one fp16 scale s and one
+ *   W2 / W3 / W4 / W8 : group-wise asymmetric uniform codes, one fp16 scale s and one
  *                  fp16 zero z (an integer) per 128-element group along K per
  *                  column; w = s * (q - z).  Sources: QFactory (ATC'25) page,
  *                  "问题与动机" and observation 1 (fine-grained asymmetric group-wise
@@ -47,8 +47,11 @@
  *     (issue them on one stream).
  *
  * Canonical (packer input) layouts, host memory:
- *   uniform codes : uint32[K / P][N], P = 32 / bits; word (j, n) bits [bits*i, bits*i + bits)
- *                   hold the code of weight (P*j + i, n)
+ *   uniform codes : uint32[K * bits / 32][N]; each column's words form one little-endian bit
+ *                   stream along K (word j = stream bits 32 j .. 32 j + 31) and the code of
+ *                   weight (k, n) is stream bits [bits*k, bits*k + bits).  For 2, 4, 8 bits:
+ *                   word (j, n) bits [bits*i, bits*i + bits) hold weight (P*j + i, n),
+ *                   P = 32 / bits; 3-bit codes (W3) straddle words, 32 codes per 3 words
  *   scales, zeros : fp16 [K / 128][N]
  *   LUT4 codes    : uint8 [K / 2][N]; low nibble = even k, high nibble = odd k
  *   LUT4 absmax   : fp32 [K / 64][N];  lut: fp16 [16]
@@ -77,7 +80,7 @@ typedef enum {
   QL_ERR_LIBRARY = 7      /* cuBLAS (prefill GEMM) could not be opened or its handle created */
 } ql_status;
 
-typedef enum { QL_FMT_W2 = 2, QL_FMT_W4 = 4, QL_FMT_W8 = 8, QL_FMT_LUT4 = 16 } ql_format;
+typedef enum { QL_FMT_W2 = 2, QL_FMT_W3 = 3, QL_FMT_W4 = 4, QL_FMT_W8 = 8, QL_FMT_LUT4 = 16 } ql_format;
 
 /* Opaque stream handle, ABI-compatible with cudaStream_t. */
 typedef struct CUstream_st* ql_stream_t;
@@ -166,6 +169,16 @@ ql_status qlinear_w2a16(const uint16_t* x, const uint32_t* qweight, const uint16
                         void* workspace, size_t workspace_bytes, ql_stream_t stream);
 
 ql_status qlinear_w8a16(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                        const uint16_t* zeros, uint16_t* y, int M, int N, int K, int group,
+                        void* workspace, size_t workspace_bytes, ql_stream_t stream);
+
+/* 3-bit codes (QFactory page, observation 1: bit widths below 4 raise the parameter share).
+ * Packed by qlinear_pack(QL_FMT_W3, ...) into two planes: the low two bits of each code
+ * where W2 puts its codes, the high bit in a separate plane (768 bytes per 16 x 128 chunk),
+ * and evaluated as sum q x = sum q2 x + 4 sum q1 x (two tensor-core steps per k-step).
+ * Arguments as qlinear_w4a16; group 128 or per-channel (group = K) only.  W3 has no prefill,
+ * policy-map or no-alloc entry. */
+ql_status qlinear_w3a16(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
                         const uint16_t* zeros, uint16_t* y, int M, int N, int K, int group,
                         void* workspace, size_t workspace_bytes, ql_stream_t stream);
 

@@ -101,7 +101,8 @@ def test_pack_tilecoo_reorders_tiles(ql):
 def test_packer_rejects_bad_shapes(ql):
     assert ql.qlinear_packed_bytes(4, 24, 128) == 0
     assert ql.qlinear_packed_bytes(4, 16, 100) == 0
-    assert ql.qlinear_packed_bytes(3, 16, 128) == 0
+    assert ql.qlinear_packed_bytes(5, 16, 128) == 0
+    assert ql.qlinear_packed_bytes(3, 16, 128) == 16 * 128 * 3 // 8
     assert ql.qlinear_packed_bytes(4, 16, 128) == 16 * 128 // 2
     assert ql._lib.qlinear_pack(4, None, None, 16, 128) == 1
     buf = np.zeros(64, dtype=np.uint8)
@@ -134,7 +135,7 @@ def test_hot_path_validates_before_any_device_work(ql):
     assert lib.qlinear_w4a16_outlier(a, a, a, a, a, a, a, a, 1, 144, 128, 128, a, 1 << 20, None) == 2
     assert lib.qlinear_w4a16_outlier(a, a, a, a, None, a, a, a, 1, 128, 128, 128, a, 1 << 20, None) == 1
     assert lib.qlinear_debug_unpack(4, None, a, 128, 128, None) == 1
-    assert lib.qlinear_debug_unpack(3, a, a, 128, 128, None) == 4
+    assert lib.qlinear_debug_unpack(5, a, a, 128, 128, None) == 4
     assert lib.qlinear_workspace_bytes(4, 0, 128, 128) == 0
 
 
@@ -231,3 +232,45 @@ def test_grouped_params_layout(ql, fmt):
     assert lib.qlinear_pack_params_grouped(16, 64, buf.ctypes.data, buf.ctypes.data, N, K) == 4
     assert lib.qlinear_pack_params_grouped(fmt, 96, buf.ctypes.data, buf.ctypes.data, N, K) == 2
     assert lib.qlinear_pack_params_grouped(fmt, 64, None, buf.ctypes.data, N, K) == 1
+
+
+def test_w3_packer_planes(ql):
+    """The W3 packer puts each code's low two bits where W2 puts a code and its high bit in the
+    second plane (word 4 + s / 4, bit 16 (dk & 1) + 4 (s % 4) + r8 / 8 + 2 (dk >> 1), after
+    the 512 bytes of quads): decoding that layout gives back the canonical codes."""
+    import oracle
+    from synth import gen
+    K, N = 384, 208
+    rs = np.random.default_rng(3)
+    codes = rs.integers(0, 8, size=(K, N), dtype=np.uint8)
+    canon = gen.pack_codes(codes, 3)
+    assert ql.qlinear_packed_bytes(3, N, K) == canon.nbytes == K * N * 3 // 8
+    packed = ql.qlinear_pack(3, canon, N, K).view(np.uint32)
+    assert np.array_equal(oracle.unpack_uniform(canon, 3), codes)
+    G, ntiles = K // 128, N // 16
+    out = np.zeros_like(codes)
+    for b in range((ntiles + 7) // 8):
+        tb = min(8, ntiles - 8 * b)
+        for g in range(G):
+            for jj in range(tb):
+                ch = packed[(b * G * 8 + g * tb + jj) * 192:][:192]
+                for lane in range(32):
+                    gi, t = lane >> 2, lane & 3
+                    w = [int(ch[lane * 4 + i]) for i in range(4)] + \
+                        [int(ch[128 + 2 * lane + i]) for i in range(2)]
+                    for s in range(8):
+                        for dk in range(4):
+                            for hi in (0, 1):
+                                k = g * 128 + 32 * (s >> 1) + 8 * t + 4 * (s & 1) + dk
+                                n = (8 * b + jj) * 16 + gi + 8 * hi
+                                # W2 position of the low bits (layout.h)
+                                q2 = (w[s >> 1] >> (16 * (dk & 1) + 8 * (dk >> 1) + 2 * hi + 4 * (s & 1))) & 3
+                                q1 = (w[4 + (s >> 2)] >> (16 * (dk & 1) + 4 * (s & 3) + hi + 2 * (dk >> 1))) & 1
+                                out[k, n] = q2 + 4 * q1
+    assert np.array_equal(out, codes)
+    lib = ql._lib
+    a = 1 << 20
+    assert lib.qlinear_w3a16(a, a, a, a, a, 1, 128, 128, 64, a, 1 << 20, None) == 2   # group 64
+    assert lib.qlinear_w3a16(None, a, a, a, a, 1, 128, 128, 128, a, 1 << 20, None) == 1
+    assert ql.qlinear_params_bytes_grouped(3, 64, N, K) == 0
+    assert ql.qlinear_params_bytes_grouped(3, K, N, K) == G * N * 2

@@ -26,8 +26,9 @@ if not os.path.exists(LIBRARY_PATH):
 
 _lib = ctypes.CDLL(LIBRARY_PATH)
 
-QL_FMT_W2, QL_FMT_W4, QL_FMT_W8, QL_FMT_LUT4 = 2, 4, 8, 16
-FORMATS = {"w2": QL_FMT_W2, "w4": QL_FMT_W4, "w8": QL_FMT_W8, "lut4": QL_FMT_LUT4}
+QL_FMT_W2, QL_FMT_W3, QL_FMT_W4, QL_FMT_W8, QL_FMT_LUT4 = 2, 3, 4, 8, 16
+FORMATS = {"w2": QL_FMT_W2, "w3": QL_FMT_W3, "w4": QL_FMT_W4, "w8": QL_FMT_W8,
+           "lut4": QL_FMT_LUT4}
 STATUS = {0: "QL_OK", 1: "QL_ERR_NULL", 2: "QL_ERR_SHAPE", 3: "QL_ERR_ALIGN",
           4: "QL_ERR_UNSUPPORTED", 5: "QL_ERR_WORKSPACE", 6: "QL_ERR_CUDA",
           7: "QL_ERR_LIBRARY"}
@@ -65,6 +66,7 @@ _SIGS = {
     "qlinear_w4a16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
     "qlinear_w2a16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
     "qlinear_w8a16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
+    "qlinear_w3a16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
     "qlinear_lut4": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
     "qlinear_w4a16_outlier": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
     "qlinear_debug_unpack": (_I, [_I, _P, _P, _I, _I, _P]),
@@ -228,6 +230,10 @@ def qlinear_w2a16(x, qweight, scales, zeros, y, M, N, K, workspace, stream=None,
 
 def qlinear_w8a16(x, qweight, scales, zeros, y, M, N, K, workspace, stream=None, group=128):
     return _uniform("qlinear_w8a16", x, qweight, scales, zeros, y, M, N, K, workspace, stream, group)
+
+
+def qlinear_w3a16(x, qweight, scales, zeros, y, M, N, K, workspace, stream=None, group=128):
+    return _uniform("qlinear_w3a16", x, qweight, scales, zeros, y, M, N, K, workspace, stream, group)
 
 
 def qlinear_w4a16_noalloc(x, qweight, scales, zeros, y, M, N, K, stream=None, group=128):

@@ -86,6 +86,12 @@ template <> struct Fmt<kW2> {
   static constexpr float kHiScale = 1.0f / 4.0f;
   static constexpr int kStagesPerWarpM8 = 2;
 };
+template <> struct Fmt<kW3> {  // low two bits as W2 codes (words 0..3), high bit in words 4, 5
+  static constexpr int kWords = 6;
+  static constexpr uint32_t kOnesHi = 0x00040004u;  // rows gi+8 carry a factor 4 (as W2)
+  static constexpr float kHiScale = 1.0f / 4.0f;
+  static constexpr int kStagesPerWarpM8 = 2;
+};
 template <> struct Fmt<kW8> {
   static constexpr int kWords = 16;
   static constexpr uint32_t kOnesHi = 0x00010001u;
@@ -120,7 +126,8 @@ struct Cfg {
   // 32 p .. 32 p + 31), so its scale and zero pairs stay in registers for those steps.
   static constexpr int NS = NS_;
   static_assert(NS == 1 || NS == 2 || NS == 4, "group 128, 64 or 32");
-  static_assert(NS == 1 || (FMT != kLUT4 && !OUTL && WPU_ == 2), "finer groups: plain uniform formats, 2 warps per unit");
+  static_assert(NS == 1 || (FMT != kLUT4 && FMT != kW3 && !OUTL && WPU_ == 2),
+                "finer groups: W2 / W4 / W8, 2 warps per unit");
   static_assert(!M1 || MT == 1, "one row of x is the M <= 8 bucket");
   static constexpr int NC = 4;                       // consumer warps
   static constexpr int WPU = WPU_;
@@ -128,7 +135,7 @@ struct Cfg {
   static constexpr int NP = NC / WPU;                // warp groups, each takes whole units
   static constexpr int kTW = kBlockTiles / WPU;      // tiles of a unit per warp
   // tiles a warp holds in registers at once (independent accumulator chains)
-  static constexpr int kQ = kTW < 4 ? kTW : (MT == 2 || FMT == kW8 || NS > 1) ? 2 : 4;
+  static constexpr int kQ = kTW < 4 ? kTW : (MT == 2 || FMT == kW8 || FMT == kW3 || NS > 1) ? 2 : 4;
   static constexpr int T = 2;                        // tiles per warp in the block epilogue
   static constexpr int kThreads = (NC + 1) * 32;     // + one producer warp
   static constexpr int KW = Fmt<FMT>::kWords;
@@ -235,6 +242,12 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
                : "r"(a));
   return v;
 }
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
@@ -403,6 +416,11 @@ struct Gemv {
         r.w[i][4 * q + 2] = v.z;
         r.w[i][4 * q + 3] = v.w;
       }
+      if constexpr (FMT == kW3) {  // the high-bit plane: 8 bytes per lane after the quads
+        const uint2 v = lds64(st + (j0 + i) * C_::kChunkBytes + 512 + lane * 8);
+        r.w[i][4] = v.x;
+        r.w[i][5] = v.y;
+      }
       if constexpr (kLut) {
         const uint4 a = lds128(st + C_::kCodeBytes + (j0 + i) * 128 + gi * 16);
         r.am[i] = make_float4(__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z),
@@ -448,6 +466,58 @@ struct Gemv {
 #pragma unroll
           for (int e = 0; e < NACC; ++e)
             if (!C_::M1 || !(e & 1)) acc[i][e] = fmaf((e & 2) ? a8 : a0, c[i][e], acc[i][e]);
+        }
+      }
+    } else if constexpr (FMT == kW3) {
+      // W3 = W2 plane (even steps in c, odd steps, which carry x16, in co) + 4 x high-bit
+      // plane (c1, every field at bit 0 of its half)
+      float c[kQ][NACC], co[kQ][NACC], c1[kQ][NACC];
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const int p = s >> 1, h = s & 1;
+        const uint32_t b0 = h ? xr[p].z : xr[p].x, b1 = h ? xr[p].w : xr[p].y;
+        uint32_t b2 = 0, b3 = 0;
+        if constexpr (MT == 2) {
+          b2 = h ? xr2[p].z : xr2[p].x;
+          b3 = h ? xr2[p].w : xr2[p].y;
+        }
+#pragma unroll
+        for (int i = 0; i < kQ; ++i) {
+          uint32_t a[4], a1[4];
+          frag_uniform<kW2>(w[i], s, a);
+          const uint32_t v1 = w[i][4 + (s >> 2)];
+#pragma unroll
+          for (int rr = 0; rr < 4; ++rr) a1[rr] = (v1 >> (4 * (s & 3) + rr)) & 0x00010001u;
+          float* cs = h ? &co[i][0] : &c[i][0];
+          if (s <= 1) {
+            hmma0(cs, a, b0, b1);
+            if constexpr (MT == 2) hmma0(cs + 4, a, b2, b3);
+          } else {
+            hmma(cs, a, b0, b1);
+            if constexpr (MT == 2) hmma(cs + 4, a, b2, b3);
+          }
+          if (s == 0) {
+            hmma0(&c1[i][0], a1, b0, b1);
+            if constexpr (MT == 2) hmma0(&c1[i][4], a1, b2, b3);
+          } else {
+            hmma(&c1[i][0], a1, b0, b1);
+            if constexpr (MT == 2) hmma(&c1[i][4], a1, b2, b3);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kQ; ++i) {
+        const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&r.p0[i]));
+        const float2 z2 = __half22float2(*reinterpret_cast<const __half2*>(&r.p1[i]));
+#pragma unroll
+        for (int e = 0; e < NACC; ++e) {
+          if (C_::M1 && (e & 1)) continue;  // batch column 1 of the fragment: no such row
+          // rows gi + 8 (e & 2) carry x4 in the W2 plane: their high bit weighs 4 x 4
+          float d = fmaf(co[i][e], 0.0625f, c[i][e]);
+          d = fmaf(c1[i][e], (e & 2) ? 16.0f : 4.0f, d);
+          const float sc = (e & 2) ? s2.y : s2.x;
+          const float zc = (e & 2) ? z2.y : z2.x;
+          acc[i][e] = fmaf(sc, fmaf(-zc, cx[e], d), acc[i][e]);
         }
       }
     } else {

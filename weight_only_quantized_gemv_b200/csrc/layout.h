@@ -34,6 +34,13 @@
 //   W8  : word 2 s + r8 / 8, bit 16 (dk & 1) + 8 (dk >> 1)
 //   LUT4: word s,            bit 16 (dk >> 1) + 8 (r8 / 8) + 4 (dk & 1)
 //         (each byte holds the two codes of one fragment register)
+//   W3  : two bit planes, q = q2 + 4 q1.  The low two bits q2 sit exactly where W2 puts a
+//         2-bit code (words 0..3, the quad of the lane); the high bit q1 sits in word
+//         4 + s / 4, bit 16 (dk & 1) + 4 (s % 4) + r8 / 8 + 2 (dk >> 1), so that shifting
+//         the word right by 4 (s % 4) + r (r = the fragment register) and masking bits
+//         0 and 16 yields register r of step s.  Words 4 and 5 of a lane are not in the
+//         quad layout: they follow the 512 bytes of quads, 8 bytes per lane (a 768-byte
+//         chunk).
 //
 // Parameters follow the chunk order: per chunk, for gi = 0..7 the pair of
 // columns (gi, gi + 8):
@@ -50,7 +57,7 @@
 
 namespace qlayout {
 
-enum { kW2 = 2, kW4 = 4, kW8 = 8, kLUT4 = 16 };
+enum { kW2 = 2, kW3 = 3, kW4 = 4, kW8 = 8, kLUT4 = 16 };
 
 constexpr int kGroup = 128;      // quantization group along K (uniform formats)
 constexpr int kLutBlock = 64;    // absmax block along K (LUT4)
@@ -59,13 +66,18 @@ constexpr int kBlockTiles = 8;   // tiles per block (128 columns)
 
 // 32-bit words of codes per lane per chunk.
 QL_HD int words_per_lane(int fmt) {
-  return fmt == kW2 ? 4 : fmt == kW8 ? 16 : 8;
+  return fmt == kW2 ? 4 : fmt == kW3 ? 6 : fmt == kW8 ? 16 : 8;
 }
 QL_HD int chunk_bytes(int fmt) { return 128 * words_per_lane(fmt); }
 QL_HD int code_bits(int fmt) { return fmt == kLUT4 ? 4 : fmt; }
 
 // 32-bit index, inside its chunk, of word w of lane l
 QL_HD int word_index(int w, int lane) { return ((w >> 2) * 32 + lane) * 4 + (w & 3); }
+
+// ... for a format: W3's high-bit words 4 and 5 follow the quads, two per lane
+QL_HD int word_index_fmt(int fmt, int w, int lane) {
+  return (fmt == kW3 && w >= 4) ? 128 + 2 * lane + (w - 4) : word_index(w, lane);
+}
 
 QL_HD int tiles_in_block(int b, int ntiles) {
   int r = ntiles - kBlockTiles * b;
@@ -100,6 +112,12 @@ QL_HD void code_position(int fmt, int s, int dk, int r8, int* word, int* bit) {
       *bit = 16 * (dk >> 1) + 8 * hi + 4 * (dk & 1);
       break;
   }
+}
+
+// W3: (word, bit) of the high bit q1 of (step s, dk, r8); q2 takes code_position(kW2, ...)
+QL_HD void code_position_w3_high(int s, int dk, int r8, int* word, int* bit) {
+  *word = 4 + (s >> 2);
+  *bit = 16 * (dk & 1) + 4 * (s & 3) + (r8 >> 3) + 2 * (dk >> 1);
 }
 
 }  // namespace qlayout

@@ -12,7 +12,9 @@ using namespace qlayout;
 
 namespace {
 
-bool fmt_ok(int fmt) { return fmt == kW2 || fmt == kW4 || fmt == kW8 || fmt == kLUT4; }
+bool fmt_ok(int fmt) {
+  return fmt == kW2 || fmt == kW3 || fmt == kW4 || fmt == kW8 || fmt == kLUT4;
+}
 
 bool shape_ok(int N, int K) {
   return N >= kTileN && K >= kGroup && N % kTileN == 0 && K % kGroup == 0;
@@ -25,11 +27,15 @@ inline uint32_t canonical_code(int fmt, const void* canon, int N, int k, int n) 
     const uint8_t v = b[(size_t)(k >> 1) * N + n];
     return (k & 1) ? (v >> 4) : (v & 0xF);
   }
+  // each column's words are one little-endian bit stream: code k in bits [b k, b k + b)
   const int bits = fmt;
-  const int P = 32 / bits;
   const uint32_t* w = static_cast<const uint32_t*>(canon);
-  const uint32_t v = w[(size_t)(k / P) * N + n];
-  return (v >> (bits * (k % P))) & ((1u << bits) - 1);
+  const long long o = (long long)bits * k;
+  const long long j = o >> 5;
+  const int sh = (int)(o & 31);
+  uint64_t v = w[(size_t)j * N + n];
+  if (sh + bits > 32) v |= (uint64_t)w[(size_t)(j + 1) * N + n] << 32;
+  return (uint32_t)(v >> sh) & ((1u << bits) - 1);
 }
 
 }  // namespace
@@ -70,10 +76,18 @@ extern "C" ql_status qlinear_pack(int fmt, const void* canonical, void* packed, 
                 const int k = g * kGroup + k_in_group(s, t, dk);
                 const int n = n_base + gi + r8;
                 int wi, bit;
-                code_position(fmt, s, dk, r8, &wi, &bit);
-                words[wi] |= canonical_code(fmt, canonical, N, k, n) << bit;
+                const uint32_t q = canonical_code(fmt, canonical, N, k, n);
+                if (fmt == kW3) {  // low two bits as a W2 code, high bit in its own plane
+                  code_position(kW2, s, dk, r8, &wi, &bit);
+                  words[wi] |= (q & 3u) << bit;
+                  code_position_w3_high(s, dk, r8, &wi, &bit);
+                  words[wi] |= (q >> 2) << bit;
+                } else {
+                  code_position(fmt, s, dk, r8, &wi, &bit);
+                  words[wi] |= q << bit;
+                }
               }
-          for (int w = 0; w < WL; ++w) chunk[word_index(w, lane)] = words[w];
+          for (int w = 0; w < WL; ++w) chunk[word_index_fmt(fmt, w, lane)] = words[w];
         }
       }
     }
@@ -152,17 +166,18 @@ static int subgroups(int group, int K) {
 }
 
 extern "C" size_t qlinear_params_bytes_grouped(int fmt, int group, int N, int K) {
-  if (fmt != kW2 && fmt != kW4 && fmt != kW8) return 0;
+  if (fmt != kW2 && fmt != kW3 && fmt != kW4 && fmt != kW8) return 0;
   if (!shape_ok(N, K) || !subgroups(group, K)) return 0;
+  if (fmt == kW3 && subgroups(group, K) != 1) return 0;  // W3: group 128 or per-channel
   return (size_t)(K / kGroup) * subgroups(group, K) * N * sizeof(uint16_t);
 }
 
 extern "C" ql_status qlinear_pack_params_grouped(int fmt, int group, const void* canonical,
                                                  void* packed, int N, int K) {
-  if (fmt != kW2 && fmt != kW4 && fmt != kW8) return QL_ERR_UNSUPPORTED;
+  if (fmt != kW2 && fmt != kW3 && fmt != kW4 && fmt != kW8) return QL_ERR_UNSUPPORTED;
   if (!canonical || !packed) return QL_ERR_NULL;
   const int NS = subgroups(group, K);
-  if (!shape_ok(N, K) || !NS) return QL_ERR_SHAPE;
+  if (!shape_ok(N, K) || !NS || (fmt == kW3 && NS != 1)) return QL_ERR_SHAPE;
   const bool per_channel = group == K && group != kGroup;
   const int G = K / kGroup;
   const int ntiles = N / kTileN;

@@ -20,7 +20,9 @@ namespace {
 constexpr int kMaxCtasPerSm = 8;
 constexpr size_t kErrBytes = 256;  // workspace[0..255]: error word (first 4 bytes)
 
-bool fmt_ok(int fmt) { return fmt == kW2 || fmt == kW4 || fmt == kW8 || fmt == kLUT4; }
+bool fmt_ok(int fmt) {
+  return fmt == kW2 || fmt == kW3 || fmt == kW4 || fmt == kW8 || fmt == kLUT4;
+}
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -94,6 +96,7 @@ KernelInfo select_kernel(int fmt, int MT, bool outl, int wpu, bool m1, bool occ2
   if (outl) return MT == 1 ? m8_kernel<kW4, true>(m1) : kernel_info<kW4, 2, true>();
   switch (fmt) {
     case kW2: return MT == 1 ? m8_kernel<kW2, false>(m1) : kernel_info<kW2, 2, false>();
+    case kW3: return MT == 1 ? m8_kernel<kW3, false>(m1) : kernel_info<kW3, 2, false>();
     case kW4:
       if (MT == 2) return kernel_info<kW4, 2, false>();
       return wpu == 4 ? w4_m8_kernel<4>(m1) : wpu == 2 ? w4_m8_kernel<2>(m1) : w4_m8_kernel<1>(m1);
@@ -397,7 +400,7 @@ __global__ void __launch_bounds__(128) debug_kernel(const uint8_t* packed, const
   uint32_t wv[KW];
   const uint32_t* src = reinterpret_cast<const uint32_t*>(packed + ch * chunk_bytes(FMT));
 #pragma unroll
-  for (int i = 0; i < KW; ++i) wv[i] = src[word_index(i, lane)];
+  for (int i = 0; i < KW; ++i) wv[i] = src[word_index_fmt(FMT, i, lane)];
   const int gi = lane >> 2, t4 = lane & 3;
   float2 s2 = make_float2(0.f, 0.f), z2 = s2;
   float4 am = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -416,7 +419,7 @@ __global__ void __launch_bounds__(128) debug_kernel(const uint8_t* packed, const
       if (DEQ) qlk::frag_lut(wv[s], (uint32_t)__cvta_generic_to_shared(tbl) + 4u * (uint32_t)lane, a);
       else a[0] = a[1] = a[2] = a[3] = 0u;
     } else {
-      qlk::frag_uniform<FMT>(wv, s, a);
+      qlk::frag_uniform<(FMT == kW3) ? kW2 : FMT>(wv, s, a);
     }
 #pragma unroll
     for (int r = 0; r < 4; ++r)
@@ -439,7 +442,9 @@ __global__ void __launch_bounds__(128) debug_kernel(const uint8_t* packed, const
         } else {
           // the fp16 value is code * 2^(shift - 24): decode it numerically
           const uint32_t iv = (uint32_t)(__half2float(hv) * 16777216.0f);
-          const uint32_t q = iv >> field_shift<FMT>(s, r);
+          uint32_t q = iv >> field_shift<(FMT == kW3) ? kW2 : FMT>(s, r);
+          if constexpr (FMT == kW3)  // high bit: bit 4 (s % 4) + r of each half of word 4 + s / 4
+            q |= ((wv[4 + (s >> 2)] >> (16 * e + 4 * (s & 3) + r)) & 1u) << 2;
           if (DEQ) {
             const float sc = (r & 1) ? s2.y : s2.x, zc = (r & 1) ? z2.y : z2.x;
             w[(size_t)k * N + n] = __fmul_rn(sc, (float)q - zc);
@@ -458,6 +463,7 @@ ql_status launch_debug(int fmt, const void* packed, const void* p0, const void* 
   const unsigned grid = (unsigned)((chunks + 3) / 4);
   switch (fmt) {
     case kW2: debug_kernel<kW2, DEQ><<<grid, 128, 0, st>>>(static_cast<const uint8_t*>(packed), p0, p1, codes, w, N, K); break;
+    case kW3: debug_kernel<kW3, DEQ><<<grid, 128, 0, st>>>(static_cast<const uint8_t*>(packed), p0, p1, codes, w, N, K); break;
     case kW4: debug_kernel<kW4, DEQ><<<grid, 128, 0, st>>>(static_cast<const uint8_t*>(packed), p0, p1, codes, w, N, K); break;
     case kW8: debug_kernel<kW8, DEQ><<<grid, 128, 0, st>>>(static_cast<const uint8_t*>(packed), p0, p1, codes, w, N, K); break;
     default: debug_kernel<kLUT4, DEQ><<<grid, 128, 0, st>>>(static_cast<const uint8_t*>(packed), p0, p1, codes, w, N, K); break;
@@ -489,7 +495,7 @@ extern "C" size_t qlinear_workspace_bytes(int fmt, int M, int N, int K) {
   Plan p;
   if (make_plan(fmt, M, N, K, false, &p) != cudaSuccess) return 0;
   // the finer-group kernels (group 64, 32) may resolve to another occupancy: cover them
-  if (fmt != kLUT4) {
+  if (fmt != kLUT4 && fmt != kW3) {
     for (int ns : {2, 4}) {
       Plan q;
       if (make_plan(fmt, M, N, K, false, &q, ns) == cudaSuccess && q.ws_bytes > p.ws_bytes)
@@ -533,6 +539,16 @@ extern "C" ql_status qlinear_plan(int fmt, int M, int N, int K, ql_plan* plan) {
 QL_UNIFORM_ENTRY(qlinear_w4a16, kW4)
 QL_UNIFORM_ENTRY(qlinear_w2a16, kW2)
 QL_UNIFORM_ENTRY(qlinear_w8a16, kW8)
+
+extern "C" ql_status qlinear_w3a16(const uint16_t* x, const uint32_t* qweight,
+                                   const uint16_t* scales, const uint16_t* zeros, uint16_t* y,
+                                   int M, int N, int K, int group, void* workspace,
+                                   size_t workspace_bytes, ql_stream_t stream) {
+  if (subgroups(group, K) != 1) return QL_ERR_SHAPE;  // group 128 or per-channel
+  Call c{kW3, false, x, qweight, scales, zeros, nullptr, nullptr, nullptr, y, M, N, K,
+         workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), 1};
+  return run(c);
+}
 
 extern "C" ql_status qlinear_lut4(const uint16_t* x, const uint8_t* codes, const uint16_t* lut16,
                                   const float* absmax, uint16_t* y, int M, int N, int K, int block,

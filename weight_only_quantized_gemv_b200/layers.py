@@ -12,15 +12,17 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (QL_FMT_LUT4, QL_FMT_W2, QL_FMT_W4, QL_FMT_W8, QL_STRATEGY_PREFILL,
+from . import (QL_FMT_LUT4, QL_FMT_W2, QL_FMT_W3, QL_FMT_W4, QL_FMT_W8, QL_STRATEGY_PREFILL,
                qlinear_debug_dequant, qlinear_policy_lookup,
                qlinear_debug_unpack, qlinear_dequant_fp16, qlinear_lut4, qlinear_pack,
                qlinear_matmul, qlinear_pack_params, qlinear_pack_params_grouped,
                qlinear_prefill,
-               qlinear_pack_tilecoo, qlinear_w2a16, qlinear_w4a16, qlinear_w4a16_outlier,
+               qlinear_pack_tilecoo, qlinear_w2a16, qlinear_w3a16, qlinear_w4a16,
+               qlinear_w4a16_outlier,
                qlinear_w8a16, qlinear_workspace_bytes)
 
-_ENTRY = {QL_FMT_W2: qlinear_w2a16, QL_FMT_W4: qlinear_w4a16, QL_FMT_W8: qlinear_w8a16}
+_ENTRY = {QL_FMT_W2: qlinear_w2a16, QL_FMT_W3: qlinear_w3a16, QL_FMT_W4: qlinear_w4a16,
+          QL_FMT_W8: qlinear_w8a16}
 
 
 def _dev(a: np.ndarray, device) -> torch.Tensor:

@@ -18,10 +18,10 @@ import json
 import torch
 
 from . import (FORMATS, QL_FMT_LUT4, qlinear_lut4, qlinear_plan, qlinear_read_error,
-               qlinear_w2a16, qlinear_w4a16, qlinear_w4a16_outlier, qlinear_w8a16,
-               qlinear_workspace_bytes)
+               qlinear_w2a16, qlinear_w3a16, qlinear_w4a16, qlinear_w4a16_outlier,
+               qlinear_w8a16, qlinear_workspace_bytes)
 
-_UNIFORM = {2: qlinear_w2a16, 4: qlinear_w4a16, 8: qlinear_w8a16}
+_UNIFORM = {2: qlinear_w2a16, 3: qlinear_w3a16, 4: qlinear_w4a16, 8: qlinear_w8a16}
 
 
 def algorithmic_bytes(fmt: int, K: int, N: int, M: int, nnz: int = 0, group: int = 128) -> int:
