@@ -42,7 +42,9 @@ Sources followed (page, section):
 Parity status: every function here is pinned by tests that do not re-state
 its formula (bounds against the unquantized weights, hand-derived golden
 fixtures, exact-integer identities, brute force on tiny inputs); see the
-``tests/test_oracle_*.py`` modules.
+``tests/test_oracle_*.py`` modules.  The comparison metric ``parity_errors``
+is pinned by hand-computed cases and planted mistakes in
+``tests/test_oracle_parity_metric.py``.
 """
 from __future__ import annotations
 
