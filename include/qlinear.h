@@ -77,7 +77,7 @@ typedef enum {
   QL_ERR_UNSUPPORTED = 4, /* unknown format */
   QL_ERR_WORKSPACE = 5,   /* workspace missing or smaller than qlinear_workspace_bytes() */
   QL_ERR_CUDA = 6,        /* a CUDA runtime call, kernel launch or cuBLAS call failed */
-  QL_ERR_LIBRARY = 7      /* cuBLAS (prefill GEMM) could not be opened or its handle created */
+  QL_ERR_LIBRARY = 7      /* reserved (no library is opened at run time) */
 } ql_status;
 
 typedef enum { QL_FMT_W2 = 2, QL_FMT_W3 = 3, QL_FMT_W4 = 4, QL_FMT_W8 = 8, QL_FMT_LUT4 = 16 } ql_format;
@@ -151,13 +151,30 @@ size_t qlinear_workspace_bytes(int fmt, int M, int N, int K);
  * `stream`, copies the word to *flags and clears it.  Synchronous. */
 ql_status qlinear_read_error(void* workspace, uint32_t* flags, ql_stream_t stream);
 
+/* Failure-detection tests of the GEMV entries' bounded waits (the QFactory page's critical
+ * analysis notes that the method leaves failure handling open; this is the library's own).
+ * Process-wide settings read by every later GEMV call:
+ *   wait_limit        : try_wait rounds after which a stage wait sets its flag
+ *                       (1 = copy landed late, 2 = stage released late) and then waits at
+ *                       most 2^22 more rounds; 0 restores the default 2^22
+ *   producer_delay_us : CTA 0's producer waits this long before its first copy
+ *   consumer_hold_us  : CTA 0's first consumer warp holds its first stage this long
+ *                       before releasing it (group-128 and per-channel kernels)
+ * Delays are at most 65535 us (QL_ERR_SHAPE otherwise); (0, 0, 0) restores normal
+ * operation.  A delay shorter than the second wait gives flagged calls with correct
+ * results.  Not thread-safe with respect to concurrent GEMV calls' settings. */
+ql_status qlinear_debug_wait_test(uint32_t wait_limit, uint32_t producer_delay_us,
+                                  uint32_t consumer_hold_us);
+
 /* ---------------------------------------------------------------------------
  * Hot path (device pointers, asynchronous on `stream`).
  *   x       : fp16 [M][K] row-major, 16-byte aligned
  *   qweight : packed codes from qlinear_pack, 32-byte aligned
- *   scales, zeros : packed fp16 parameters from qlinear_pack_params, 4-byte aligned
+ *   scales, zeros : packed fp16 parameters from qlinear_pack_params (group 128) or
+ *             qlinear_pack_params_grouped (group 64, 32 or K), 16-byte aligned
  *   y       : fp16 [M][N] row-major output (round-to-nearest-even of an fp32 sum)
- *   group   : must be 128
+ *   group   : W2 / W4 / W8: 128, 64, 32 or K (per-channel); W3: 128 or K; the outlier
+ *             variant and qlinear_w4a16_noalloc: 128 (QL_ERR_SHAPE otherwise)
  * ------------------------------------------------------------------------- */
 
 ql_status qlinear_w4a16(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
@@ -213,12 +230,21 @@ ql_status qlinear_w4a16_outlier(const uint16_t* x, const uint32_t* qweight,
  * 8 MiB array inside the library (on every device, from library load to process exit).
  * It allocates nothing and frees nothing.  Returns QL_ERR_WORKSPACE if a call would need
  * more than that scratch.  The first call on a device looks up the scratch's device
- * address (make it before any stream capture).  Every call on a device shares the
- * scratch: calls whose device work overlaps in time race and must not be issued;
- * each call clears the parts that must start at zero on `stream` before its launch. */
+ * address (make it before any stream capture); it is looked up again when the device's
+ * context changes (a device reset may move the array).  Every call on a device shares
+ * the scratch: calls whose device work overlaps in time race and must not be issued.
+ * Each call clears its arrival counters on `stream` before its launch, after every
+ * argument check (a rejected call enqueues nothing).  A device wait that gives up sets
+ * a flag in the scratch's error word, which stays set until
+ * qlinear_w4a16_noalloc_read_error reads it. */
 ql_status qlinear_w4a16_noalloc(const uint16_t* x, const uint32_t* qweight,
                                 const uint16_t* scales, const uint16_t* zeros, uint16_t* y,
                                 int M, int N, int K, int group, ql_stream_t stream);
+
+/* The error word of qlinear_w4a16_noalloc's scratch on the current device (the flags of
+ * qlinear_read_error), then cleared.  Waits for `stream`; synchronous.  Allocates
+ * nothing.  No page describes this entry; it has no counterpart in the method. */
+ql_status qlinear_w4a16_noalloc_read_error(uint32_t* flags, ql_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Prefill (M >> 16): stand-alone dequantization to fp16, then one dense GEMM.
@@ -244,16 +270,29 @@ ql_status qlinear_dequant_fp16(int fmt, const void* packed, const void* p0, cons
                                uint16_t* w, int N, int K, ql_stream_t stream);
 
 /* y[M][N] = x[M][K] . w_fp16[N][K]^T for any M >= 1: qlinear_dequant_fp16 into the caller's
- * w_fp16 (N * K * 2 bytes, 16-byte aligned, overwritten), then one cuBLAS GEMM on `stream`
- * (fp16 operands and output, fp32 accumulation).  x and y are fp16 row-major device arrays
- * (2-byte aligned; 16-byte alignment is faster).  cuBLAS is opened at run time
- * (libcublas.so.12); the first call on a thread and device creates a cuBLAS handle, which
- * allocates cuBLAS's own device memory and is kept for the life of the process: make that
- * first call outside stream capture.  Returns QL_ERR_LIBRARY when cuBLAS cannot be opened
- * or the handle cannot be created, QL_ERR_CUDA when the GEMM fails. */
+ * w_fp16 (N * K * 2 bytes, 16-byte aligned, overwritten), then this library's tensor-core
+ * GEMM on `stream` (tcgen05.mma with fp16 operands staged by TMA, fp32 accumulation in
+ * tensor memory, fp16 round-to-nearest-even output).  x is an fp16 row-major device array,
+ * 16-byte aligned (QL_ERR_ALIGN otherwise); y fp16 row-major, 2-byte aligned.  N % 16 == 0,
+ * K % 128 == 0.  Device waits that run out are reported by qlinear_prefill_read_error. */
 ql_status qlinear_prefill(int fmt, const uint16_t* x, const void* packed, const void* p0,
                           const void* p1, uint16_t* w_fp16, uint16_t* y, int M, int N, int K,
                           ql_stream_t stream);
+
+/* The same product without the fp16 weight matrix: y[M][N] = x[M][K] . W^T with W the fp16
+ * weights qlinear_dequant_fp16 would write, dequantized inside the GEMM (the NF4 page's
+ * codes -> FP16 -> matmul, with FP16 kept in shared memory as the tensor cores' operand
+ * instead of written back).  fmt W2 / W4 / W8 (group 128) or LUT4; packed, p0, p1 as for
+ * qlinear_dequant_fp16; x 16-byte aligned, y 2-byte aligned; any M >= 1, N % 16 == 0,
+ * K % 128 == 0.  Asynchronous on `stream`; allocates nothing. */
+ql_status qlinear_prefill_fused(int fmt, const uint16_t* x, const void* packed, const void* p0,
+                                const void* p1, uint16_t* y, int M, int N, int K,
+                                ql_stream_t stream);
+
+/* Sticky flags of the prefill GEMM kernels' bounded waits on the current device (1: a
+ * pipeline stage's wait ran out, 2: an accumulator's wait ran out; results of such a call
+ * are undefined), then cleared.  Waits for `stream`; synchronous. */
+ql_status qlinear_prefill_read_error(uint32_t* flags, ql_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Codebook GEMV with a Psumbook.  Source: CodeGEMM page (NeurIPS 2025 notes), method:

@@ -38,6 +38,7 @@ def _cols(N, seed, n=192):
 def _run(lay, x):
     y = lay.forward(torch.from_numpy(x).to(DEV))
     torch.cuda.synchronize()
+    assert lay.read_error() == 0, "a device wait gave up"
     return y.float().cpu().numpy()
 
 

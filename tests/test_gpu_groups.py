@@ -37,6 +37,7 @@ def _layer(seed, K, N, bits, group):
 def _run(lay, x):
     y = lay.forward(torch.from_numpy(x).to(DEV))
     torch.cuda.synchronize()
+    assert lay.read_error() == 0, "a device wait gave up"
     return y.float().cpu().numpy()
 
 

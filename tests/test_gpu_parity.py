@@ -44,6 +44,13 @@ def _np(t):
     return t.float().cpu().numpy()
 
 
+def _fwd(lay, xd):
+    """lay.forward, then the check that every device wait of the call completed."""
+    y = _np(lay.forward(xd))
+    assert lay.read_error() == 0, "a device wait gave up"
+    return y
+
+
 # ---------------------------------------------------------------------------
 # decode, bit-exact
 
@@ -83,7 +90,7 @@ def test_uniform_gemv_parity(name, bits, K, N, M):
     u = uniform_layer(200 + bits, K, N, bits)
     lay = layers.from_uniform(u, DEV)
     x, xd = _x(200 + M, M, K)
-    y = _np(lay.forward(xd))
+    y = _fwd(lay, xd)
     assert_parity(y, oracle.gemv_uniform(x, u.qweight, u.scales, u.zeros, bits, 128),
                   what=f"{name} M={M} K={K} N={N}")
 
@@ -94,7 +101,7 @@ def test_lut4_gemv_parity(K, N, M):
     lt = lut4_layer(400, K, N)
     lay = layers.from_lut4(lt, DEV)
     x, xd = _x(400 + M, M, K)
-    y = _np(lay.forward(xd))
+    y = _fwd(lay, xd)
     assert_parity(y, oracle.gemv_lut4(x, lt.qbytes, lt.lut, lt.absmax, 64), what=f"lut4 M={M}")
 
 
@@ -104,7 +111,7 @@ def test_outlier_gemv_parity(K, N, M):
     o = outlier_layer(500, K, N)
     lay = layers.from_outlier(o, DEV)
     x, xd = _x(500 + M, M, K)
-    y = _np(lay.forward(xd))
+    y = _fwd(lay, xd)
     ref = oracle.gemv_outlier(x, o.dense.qweight, o.dense.scales, o.dense.zeros, o.tile_offsets,
                               o.tile_rc, o.tile_vals, 4, 128)
     assert_parity(y, ref, what=f"outlier M={M} K={K} N={N}")
@@ -138,7 +145,7 @@ def test_split_k_partitions(kind, cap):
         assert ql.qlinear_plan(4, M, N, K).ctas == min(int(cap), (N // 128 + 1) * (K // 128)) \
             or kind != "w4"
         for _ in range(2):  # the second call checks that the counters were reset
-            y = _np(lay.forward(xd))
+            y = _fwd(lay, xd)
             assert_parity(y, ref, what=f"{kind} cap={cap}")
     finally:
         if old is None:
@@ -164,7 +171,7 @@ def test_w4_warps_per_unit(wpu, cap, M):
         ref = oracle.gemv_uniform(x, u.qweight, u.scales, u.zeros, 4, 128)
         assert ql.qlinear_plan(4, M, N, K).warps_per_unit == int(wpu)
         for _ in range(2):
-            assert_parity(_np(lay.forward(xd)), ref, what=f"w4 wpu={wpu} cap={cap} M={M}")
+            assert_parity(_fwd(lay, xd), ref, what=f"w4 wpu={wpu} cap={cap} M={M}")
     finally:
         for k, v in old.items():
             if v is None:
@@ -226,7 +233,7 @@ def test_codes_at_zero_point_cancel_and_outlier_only_is_exact():
     # The deferred form computes sum_k z x - z sum_k x: it cancels up to fp32 rounding of the
     # two sums (eager dequantization would give exact zeros).  Bound: a few fp32 ulps of
     # s * z * sum_k |x| per group.
-    y = _np(dense.forward(xd))
+    y = _fwd(dense, xd)
     s = d.scales.astype(np.float64)
     z = d.zeros.astype(np.float64)
     xa = np.abs(x.astype(np.float64)).reshape(5, K // 128, 128).sum(axis=2)

@@ -35,6 +35,7 @@ def _layer(seed, K, N, group=128):
 def _run(lay, x):
     y = lay.forward(torch.from_numpy(x).to(DEV))
     torch.cuda.synchronize()
+    assert lay.read_error() == 0, "a device wait gave up"
     return y.float().cpu().numpy()
 
 

@@ -73,9 +73,13 @@ _SIGS = {
     "qlinear_debug_dequant": (_I, [_I, _P, _P, _P, _P, _I, _I, _P]),
     "qlinear_plan": (_I, [_I, _I, _I, _I, ctypes.POINTER(ql_plan)]),
     "qlinear_read_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint32), _P]),
+    "qlinear_debug_wait_test": (_I, [ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint32]),
     "qlinear_w4a16_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "qlinear_w4a16_noalloc_read_error": (_I, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "qlinear_dequant_fp16": (_I, [_I, _P, _P, _P, _P, _I, _I, _P]),
     "qlinear_prefill": (_I, [_I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "qlinear_prefill_fused": (_I, [_I, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "qlinear_prefill_read_error": (_I, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "qlinear_policy_set": (_I, [ctypes.POINTER(ql_policy_entry), _I]),
     "qlinear_policy_size": (_I, []),
     "qlinear_policy_lookup": (_I, [_I, _I, _I, _I, ctypes.POINTER(ql_policy_entry),
@@ -200,6 +204,12 @@ def qlinear_plan(fmt: int, M: int, N: int, K: int) -> ql_plan:
     return p
 
 
+def qlinear_debug_wait_test(wait_limit=0, producer_delay_us=0, consumer_hold_us=0) -> None:
+    """Settings for tests of the bounded device waits; no arguments restores the defaults."""
+    _check(_lib.qlinear_debug_wait_test(wait_limit, producer_delay_us, consumer_hold_us),
+           "qlinear_debug_wait_test")
+
+
 def qlinear_read_error(workspace, stream=None) -> int:
     """Sticky error flags of the calls that used `workspace` (then cleared); 0 = none."""
     flags = ctypes.c_uint32(0)
@@ -241,6 +251,15 @@ def qlinear_w4a16_noalloc(x, qweight, scales, zeros, y, M, N, K, stream=None, gr
     _check(_lib.qlinear_w4a16_noalloc(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(y),
                                       M, N, K, group, _stream(stream)), "qlinear_w4a16_noalloc")
     return y
+
+
+def qlinear_w4a16_noalloc_read_error(stream=None) -> int:
+    """Sticky error flags of qlinear_w4a16_noalloc's scratch on the current device (then
+    cleared); 0 = none."""
+    flags = ctypes.c_uint32(0)
+    _check(_lib.qlinear_w4a16_noalloc_read_error(ctypes.byref(flags), _stream(stream)),
+           "qlinear_w4a16_noalloc_read_error")
+    return int(flags.value)
 
 
 def qlinear_lut4(x, codes, lut16, absmax, y, M, N, K, workspace, stream=None, block=64):
@@ -286,6 +305,22 @@ def qlinear_prefill(fmt, x, packed, p0, p1, w_fp16, y, M, N, K, stream=None):
     _check(_lib.qlinear_prefill(fmt, _ptr(x), _ptr(packed), _ptr(p0), _ptr(p1), _ptr(w_fp16),
                                 _ptr(y), M, N, K, _stream(stream)), "qlinear_prefill")
     return y
+
+
+def qlinear_prefill_fused(fmt, x, packed, p0, p1, y, M, N, K, stream=None):
+    """``y[M, N] = x[M, K] @ W^T`` with the weights dequantized inside the tensor-core GEMM."""
+    _check(_lib.qlinear_prefill_fused(fmt, _ptr(x), _ptr(packed), _ptr(p0), _ptr(p1), _ptr(y),
+                                      M, N, K, _stream(stream)), "qlinear_prefill_fused")
+    return y
+
+
+def qlinear_prefill_read_error(stream=None) -> int:
+    """Sticky wait-timeout flags of the prefill GEMM kernels on the current device (then
+    cleared); 0 = none."""
+    flags = ctypes.c_uint32(0)
+    _check(_lib.qlinear_prefill_read_error(ctypes.byref(flags), _stream(stream)),
+           "qlinear_prefill_read_error")
+    return int(flags.value)
 
 
 # ---------------------------------------------------------------------------

@@ -16,8 +16,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libqlinear.so")
 
-SOURCES = ["qlinear.cu", "dequant.cu", "codebook.cu", "policy.cpp", "pack.cpp"]
-HEADERS = ["kernels.cuh", "layout.h", "policy.h"]
+SOURCES = ["qlinear.cu", "dequant.cu", "prefill_tc.cu", "codebook.cu", "policy.cpp", "pack.cpp"]
+HEADERS = ["kernels.cuh", "layout.h", "policy.h", "dequant_frag.cuh"]
 
 
 def nvcc_path() -> str:

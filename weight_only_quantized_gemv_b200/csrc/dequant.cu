@@ -14,19 +14,18 @@
 // of one column (the packed fragment order), so it writes them as one 16-byte store; a
 // warp store covers 8 rows x 64 contiguous bytes, whole 32-byte sectors.
 //
-// The dense GEMM is cuBLAS (opened at run time with dlopen, so loading this library needs
-// neither cuBLAS nor a GPU): y[M][N] = x[M][K] . W[N][K]^T, fp16 in and out, fp32
-// accumulation.
+// The dense GEMM is this library's tcgen05 kernel (prefill_tc.cu): y[M][N] = x[M][K] .
+// W[N][K]^T, fp16 in and out, fp32 accumulation.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
-#include <cublas_v2.h>  // types and prototypes only; the library is opened with dlopen
-#include <dlfcn.h>
 
-#include <mutex>
-#include <unordered_map>
-
+#include "dequant_frag.cuh"
 #include "layout.h"
 #include "qlinear.h"
+
+// the tensor-core GEMM of prefill_tc.cu
+ql_status qlinear_gemm_f16_tc(const uint16_t* x, const uint16_t* w, uint16_t* y, int M, int N,
+                              int K, cudaStream_t st);
 
 using namespace qlayout;
 
@@ -50,99 +49,33 @@ __device__ __forceinline__ void stg128(void* p, uint32_t a, uint32_t b, uint32_t
                : "memory");
 }
 
-__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) {
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) {
-  return *reinterpret_cast<__half2*>(&u);
-}
-
-// Bit offset (inside each 16-bit half of fragment register r of step s) of the code field
-// that the AND masks below leave in place.
-template <int FMT>
-__device__ __forceinline__ constexpr int field_shift(int s, int r) {
-  return FMT == kW4 ? ((r & 1) ? 4 : 0) : FMT == kW2 ? 4 * (s & 1) + ((r & 1) ? 2 : 0) : 0;
-}
-
-// The code fields of fragment register r of step s, each in its own 16-bit half (low half =
-// the smaller k), at the bit offsets field_shift() gives.
-template <int FMT>
-__device__ __forceinline__ uint32_t code_fields(const uint32_t* w, int s, int r) {
-  if constexpr (FMT == kW4) {
-    const uint32_t v = (r >> 1) ? (w[s] >> 8) : w[s];
-    return v & ((r & 1) ? 0x00F000F0u : 0x000F000Fu);
-  } else if constexpr (FMT == kW2) {
-    const uint32_t v = (r >> 1) ? (w[s >> 1] >> 8) : w[s >> 1];
-    const uint32_t m = (r & 1) ? ((s & 1) ? 0x00C000C0u : 0x000C000Cu)
-                               : ((s & 1) ? 0x00300030u : 0x00030003u);
-    return v & m;
-  } else {  // W8: words 2s (rows gi) and 2s + 1 (rows gi + 8)
-    const uint32_t v = (r >> 1) ? (w[2 * s + (r & 1)] >> 8) : w[2 * s + (r & 1)];
-    return v & 0x00FF00FFu;
-  }
-}
-
-// fp16 bit pattern of 2^(10 - sh): its last mantissa bit weighs 2^-sh, so OR-ing a code
-// field that sits at bit offset sh into the mantissa gives exactly 2^(10 - sh) + q.
-__device__ __forceinline__ constexpr uint32_t magic_half(int sh) {
-  return (uint32_t)(25 - sh) << 10;
-}
-
-// W2 / W4 / W8: w = fp16(s * (q - z)).  (2^(10-sh) + q) - (2^(10-sh) + z) = q - z is exact
-// in fp16 (|q - z| <= 255 < 2^11), and the fp16 product rounds the exact s (q - z) once.
+// W2 / W4 / W8: a lane's 64 weights of the chunk, fp16(s * (q - z)) (dequant_frag.cuh).
 template <int FMT>
 __device__ __forceinline__ void dequant_chunk_uniform(const uint32_t* wv, __half2 s_lo,
                                                       __half2 s_hi, float z_lo, float z_hi,
                                                       __half* out_lo, __half* out_hi) {
-  // z + 2^(10 - sh) per (step parity, row half): exact small integers / dyadics in fp16
   __half2 zb[2][2];
-#pragma unroll
-  for (int p = 0; p < 2; ++p)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int sh = field_shift<FMT>(p, h);
-      zb[p][h] = __float2half2_rn((float)(1 << (10 - sh)) + (h ? z_hi : z_lo));
-    }
+  qdq::zero_bias<FMT>(z_lo, z_hi, zb);
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      uint32_t o[4];
-#pragma unroll
-      for (int ss = 0; ss < 2; ++ss)
-#pragma unroll
-        for (int dkp = 0; dkp < 2; ++dkp) {
-          const int s = 2 * i + ss, r = h + 2 * dkp;
-          const uint32_t f = code_fields<FMT>(wv, s, r) | (magic_half(field_shift<FMT>(s, r)) * 0x10001u);
-          const __half2 d = __hsub2(u32_as_h2(f), zb[s & 1][h]);
-          o[2 * ss + dkp] = h2_as_u32(__hmul2(d, h ? s_hi : s_lo));
-        }
-      stg128((h ? out_hi : out_lo) + 32 * i, o[0], o[1], o[2], o[3]);
+      const uint4 o = qdq::uniform_pair8<FMT>(wv, 2 * i, h, zb, h ? s_hi : s_lo);
+      stg128((h ? out_hi : out_lo) + 32 * i, o.x, o.y, o.z, o.w);
     }
 }
 
-// LUT4: w = fp16(fp32(lut[q]) * absmax) with the product rounded to fp32 first.  Byte r of
-// word s holds the two codes of fragment register r (low nibble = the smaller k).
+// LUT4: a lane's 64 weights of the chunk, fp16(fp32(lut[q]) * absmax).  am = the absmax of
+// (rows gi, gi + 8) for k < 64 and (rows gi, gi + 8) for k >= 64.
 __device__ __forceinline__ void dequant_chunk_lut4(const uint32_t* wv, const float* lut_s,
                                                    float4 am, __half* out_lo, __half* out_hi) {
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      uint32_t o[4];
-#pragma unroll
-      for (int ss = 0; ss < 2; ++ss)
-#pragma unroll
-        for (int dkp = 0; dkp < 2; ++dkp) {
-          const int s = 2 * i + ss, r = h + 2 * dkp;
-          // absmax block: k in the group < 64 for steps 0..3; (x, y) = rows (gi, gi + 8)
-          const float a = (s >= 4) ? (h ? am.w : am.z) : (h ? am.y : am.x);
-          const uint32_t byte = (wv[s] >> (8 * r)) & 0xFFu;
-          const float lo = __fmul_rn(lut_s[byte & 0xFu], a);
-          const float hi = __fmul_rn(lut_s[byte >> 4], a);
-          o[2 * ss + dkp] = h2_as_u32(__floats2half2_rn(lo, hi));
-        }
-      stg128((h ? out_hi : out_lo) + 32 * i, o[0], o[1], o[2], o[3]);
+      const float a = (i >= 2) ? (h ? am.w : am.z) : (h ? am.y : am.x);
+      const uint4 o = qdq::lut_pair8(wv, 2 * i, h, lut_s, a);
+      stg128((h ? out_hi : out_lo) + 32 * i, o.x, o.y, o.z, o.w);
     }
 }
 
@@ -218,50 +151,6 @@ ql_status launch_dequant(int fmt, const void* packed, const void* p0, const void
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
-// ---------------------------------------------------------------------------
-// cuBLAS, opened at run time
-
-// the C symbol cublasGemmEx (C++ also sees an inline overload taking cudaDataType)
-using GemmEx = cublasStatus_t (*)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int,
-                                  int, const void*, const void*, cudaDataType, int, const void*,
-                                  cudaDataType, int, const void*, void*, cudaDataType, int,
-                                  cublasComputeType_t, cublasGemmAlgo_t);
-
-struct Blas {
-  decltype(&cublasCreate_v2) create = nullptr;
-  decltype(&cublasSetStream_v2) set_stream = nullptr;
-  GemmEx gemm = nullptr;
-  bool ok = false;
-};
-
-const Blas& blas() {
-  static Blas b;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* h = dlopen("libcublas.so.12", RTLD_NOW | RTLD_GLOBAL);
-    if (!h) h = dlopen("libcublas.so", RTLD_NOW | RTLD_GLOBAL);
-    if (!h) return;
-    b.create = reinterpret_cast<decltype(&cublasCreate_v2)>(dlsym(h, "cublasCreate_v2"));
-    b.set_stream = reinterpret_cast<decltype(&cublasSetStream_v2)>(dlsym(h, "cublasSetStream_v2"));
-    b.gemm = reinterpret_cast<GemmEx>(dlsym(h, "cublasGemmEx"));
-    b.ok = b.create && b.set_stream && b.gemm;
-  });
-  return b;
-}
-
-// One handle per (thread, device), created on first use and kept for the process.
-cublasHandle_t blas_handle(const Blas& b) {
-  thread_local std::unordered_map<int, cublasHandle_t> handles;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-  auto it = handles.find(dev);
-  if (it != handles.end()) return it->second;
-  cublasHandle_t h = nullptr;
-  if (b.create(&h) != CUBLAS_STATUS_SUCCESS) return nullptr;
-  handles.emplace(dev, h);
-  return h;
-}
-
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -283,20 +172,9 @@ extern "C" ql_status qlinear_prefill(int fmt, const uint16_t* x, const void* pac
   ql_status st = check_dequant(fmt, packed, p0, p1, w_fp16, N, K);
   if (st != QL_OK) return st;
   if (M <= 0) return QL_ERR_SHAPE;
-  if (!aligned(x, 2) || !aligned(y, 2)) return QL_ERR_ALIGN;
-  const Blas& b = blas();
-  if (!b.ok) return QL_ERR_LIBRARY;
-  cublasHandle_t h = blas_handle(b);
-  if (!h) return QL_ERR_LIBRARY;
+  if (!aligned(x, 16) || !aligned(y, 2)) return QL_ERR_ALIGN;
   const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   st = launch_dequant(fmt, packed, p0, p1, w_fp16, N, K, cs);
   if (st != QL_OK) return st;
-  if (b.set_stream(h, cs) != CUBLAS_STATUS_SUCCESS) return QL_ERR_LIBRARY;
-  const float one = 1.0f, zero = 0.0f;
-  // column-major view: y^T (N x M, ld N) = W^T (op T of the K x N view of W[N][K], ld K)
-  //                                        . x^T (K x M view of x[M][K], ld K)
-  const cublasStatus_t cs2 = b.gemm(h, CUBLAS_OP_T, CUBLAS_OP_N, N, M, K, &one, w_fp16, CUDA_R_16F,
-                                    K, x, CUDA_R_16F, K, &zero, y, CUDA_R_16F, N,
-                                    CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
-  return cs2 == CUBLAS_STATUS_SUCCESS ? QL_OK : QL_ERR_CUDA;
+  return qlinear_gemm_f16_tc(x, w_fp16, y, M, N, K, cs);
 }

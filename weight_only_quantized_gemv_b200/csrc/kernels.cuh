@@ -37,9 +37,10 @@
 //  * The outlier variant adds the Tile-COO entries of each unit into a shared fp32
 //    y tile, reading x from the same stage the dense path uses; the y tile joins
 //    the dense sums at the end of the unit range, before the split-K fix-up.
-//  * Every mbarrier wait is bounded.  A wait that runs out sets a bit in the
-//    workspace error word and carries on, so a lost copy can corrupt results but
-//    never hang the GPU.
+//  * Every mbarrier wait is bounded.  A wait that passes its limit sets a bit in the
+//    workspace error word, then waits at most as long again for the late copy (or the
+//    late release) and carries on; a lost copy can corrupt results but never hang the
+//    GPU, and every copy a CTA issued has landed when it exits unless a wait gave up.
 #pragma once
 #include <cuda.h>  // CUtensorMap
 #include <cuda_fp16.h>
@@ -71,6 +72,11 @@ struct GemvParams {
   int M, N, K, G, nblocks, ntiles;
   int U;                      // nblocks * G
   int C;                      // CTAs
+  uint32_t wait_limit;        // try_wait rounds before a wait is flagged (kSpinLimit)
+  // tests of the bounded waits only (0 otherwise): bits 0-15 delay CTA 0's producer before
+  // its first copy, bits 16-31 hold CTA 0's consumer warp 0 before it releases its first
+  // stage, in microseconds
+  uint32_t test_us;
 };
 
 template <int FMT> struct Fmt;
@@ -196,8 +202,8 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 }
 
 // Bounded wait for the phase with parity `parity` to complete; false if abandoned.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  for (uint32_t it = 0; it < kSpinLimit; ++it) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit) {
+  for (uint32_t it = 0; it < limit; ++it) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -209,6 +215,29 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     if (done) return true;
   }
   return false;
+}
+
+// Wait for a stage's phase.  Past P.wait_limit rounds the wait sets `bit` in the error
+// word and goes on waiting for at most kSpinLimit more rounds (a late copy still lands
+// before it is read); if it then gives up too, the results are undefined.
+__device__ __forceinline__ void stage_wait(const GemvParams& P, uint32_t bar, uint32_t parity,
+                                           uint32_t bit) {
+  if (!mbar_wait(bar, parity, P.wait_limit)) {
+    atomicOr(P.err, bit);
+    mbar_wait(bar, parity, kSpinLimit);
+  }
+}
+
+// Tests of the bounded waits: let `us` microseconds pass (a fixed, bounded delay).
+__device__ __forceinline__ void test_delay(uint32_t us) {
+  uint64_t t0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  for (;;) {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (t - t0 >= 1000ull * us) return;
+    __nanosleep(1000);
+  }
 }
 
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
@@ -768,6 +797,7 @@ struct Gemv {
             : "memory");
       }
     };
+    if ((P.test_us & 0xFFFFu) && blockIdx.x == 0) test_delay(P.test_us & 0xFFFFu);
     const int b0 = u0 / P.G, g0 = u0 - b0 * P.G;
     int b = b0, g = g0;
     const int pre = n < S ? n : S;
@@ -783,7 +813,7 @@ struct Gemv {
     g = g0;
     for (int i = 0; i < n; ++i) {
       if (i >= S) {
-        if (!mbar_wait(bars + 8 * (S + i % S), ((i / S) - 1) & 1)) atomicOr(P.err, kErrEmptyTimeout);
+        stage_wait(P, bars + 8 * (S + i % S), ((i / S) - 1) & 1, kErrEmptyTimeout);
         weights(i, b, g);
       }
       activations(i, g);
@@ -812,7 +842,7 @@ struct Gemv {
     const int s = i % S;
     const int tb = tiles_in_block(b, P.ntiles);
     const uint32_t st = ring + s * C_::kStageBytes;
-    if (!mbar_wait(bars + 8 * s, (i / S) & 1)) atomicOr(P.err, kErrFullTimeout);
+    stage_wait(P, bars + 8 * s, (i / S) & 1, kErrFullTimeout);
     uint4 xr[4], xr2[4];
     read_x(P, st, lane, xr, xr2);
     if constexpr (OUTL) {
@@ -993,7 +1023,7 @@ struct Gemv {
     const int s = i % S;
     const int tb = tiles_in_block(b, P.ntiles);
     const uint32_t st = ring + s * C_::kStageBytes;
-    if (!mbar_wait(bars + 8 * s, (i / S) & 1)) atomicOr(P.err, kErrFullTimeout);
+    stage_wait(P, bars + 8 * s, (i / S) & 1, kErrFullTimeout);
     uint4 xr[4], xr2[4];
     read_x(P, st, lane, xr, xr2);
     const int t0 = kTW * sub;
@@ -1064,6 +1094,12 @@ struct Gemv {
 #pragma unroll
       for (int e = 0; e < NACC; ++e) acc[j][e] = 0.f;
     uint32_t orc[3] = {0, 0, 0}, oval[3] = {0, 0, 0};
+    // tests of the bounded waits: CTA 0's warp 0 takes stage 0 and holds it for a while
+    // before its first unit releases it (waiting for a completed phase again returns at once)
+    if ((P.test_us >> 16) && blockIdx.x == 0 && warp == 0 && n > 0) {
+      stage_wait(P, smem_addr(smem) + C_::kBarOff, 0, kErrFullTimeout);
+      test_delay(P.test_us >> 16);
+    }
     if constexpr (OUTL) {
       consumer_sync(NC * 32);  // the Tile-COO offsets are in shared memory
       prefetch_outliers(P, reinterpret_cast<const uint32_t*>(smem + C_::kToffOff), grp, n,

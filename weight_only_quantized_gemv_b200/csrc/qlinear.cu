@@ -6,6 +6,7 @@
 #include <stdint.h>
 #include <stdlib.h>
 
+#include <atomic>
 #include <mutex>
 #include <unordered_map>
 
@@ -19,6 +20,10 @@ namespace {
 
 constexpr int kMaxCtasPerSm = 8;
 constexpr size_t kErrBytes = 256;  // workspace[0..255]: error word (first 4 bytes)
+
+// Settings of qlinear_debug_wait_test (tests of the bounded waits; defaults otherwise).
+std::atomic<uint32_t> g_wait_limit{qlk::kSpinLimit};
+std::atomic<uint32_t> g_test_us{0};
 
 bool fmt_ok(int fmt) {
   return fmt == kW2 || fmt == kW3 || fmt == kW4 || fmt == kW8 || fmt == kLUT4;
@@ -306,7 +311,8 @@ int subgroups(int group, int K) {
   return 0;
 }
 
-ql_status run(const Call& c) {
+// Argument checks that need no device state (pointers, shapes, alignment).
+ql_status check_call(const Call& c) {
   if (!c.x || !c.qw || !c.p0 || !c.p1 || !c.y) return QL_ERR_NULL;
   if (c.outl && (!c.toff || !c.trc || !c.tval)) return QL_ERR_NULL;
   if (!shape_ok(c.M, c.N, c.K)) return QL_ERR_SHAPE;
@@ -320,6 +326,12 @@ ql_status run(const Call& c) {
   }
   if (c.outl && (!aligned(c.toff, 4) || !aligned(c.trc, 2) || !aligned(c.tval, 2)))
     return QL_ERR_ALIGN;
+  return QL_OK;
+}
+
+ql_status run(const Call& c) {
+  const ql_status chk = check_call(c);
+  if (chk != QL_OK) return chk;
   Plan p;
   if (make_plan(c.fmt, c.M, c.N, c.K, c.outl, &p, c.ns) != cudaSuccess) return QL_ERR_CUDA;
   if (!c.ws || c.ws_bytes < p.ws_bytes) return QL_ERR_WORKSPACE;
@@ -344,6 +356,8 @@ ql_status run(const Call& c) {
   P.ntiles = p.ntiles;
   P.U = (int)p.U;
   P.C = p.C;
+  P.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
+  P.test_us = g_test_us.load(std::memory_order_relaxed);
   const KernelInfo k = select_kernel(c.fmt, p.MT, c.outl, p.WPU, p.M1, p.OCC2, p.NS);
   // Programmatic stream serialization: the kernel may start while the previous kernel in
   // the stream drains; it requests only static weight bytes before griddepcontrol.wait.
@@ -480,7 +494,7 @@ extern "C" const char* ql_status_str(int status) {
   switch (status) {
     case QL_OK: return "ok";
     case QL_ERR_NULL: return "null pointer argument";
-    case QL_ERR_SHAPE: return "unsupported shape (M in 1..16, N % 16 == 0, K % 128 == 0, group 128, block 64)";
+    case QL_ERR_SHAPE: return "unsupported shape (M in 1..16, N % 16 == 0, K % 128 == 0, group 128 / 64 / 32 / K, block 64)";
     case QL_ERR_ALIGN: return "misaligned pointer";
     case QL_ERR_UNSUPPORTED: return "unknown format";
     case QL_ERR_WORKSPACE: return "workspace missing or too small";
@@ -593,6 +607,14 @@ extern "C" ql_status qlinear_debug_dequant(int fmt, const void* packed, const vo
                             reinterpret_cast<cudaStream_t>(stream));
 }
 
+extern "C" ql_status qlinear_debug_wait_test(uint32_t wait_limit, uint32_t producer_delay_us,
+                                             uint32_t consumer_hold_us) {
+  if (producer_delay_us > 0xFFFFu || consumer_hold_us > 0xFFFFu) return QL_ERR_SHAPE;
+  g_wait_limit.store(wait_limit ? wait_limit : qlk::kSpinLimit, std::memory_order_relaxed);
+  g_test_us.store(producer_delay_us | (consumer_hold_us << 16), std::memory_order_relaxed);
+  return QL_OK;
+}
+
 extern "C" ql_status qlinear_read_error(void* workspace, uint32_t* flags, ql_stream_t stream) {
   if (!workspace || !flags) return QL_ERR_NULL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -614,11 +636,14 @@ extern "C" ql_status qlinear_read_error(void* workspace, uint32_t* flags, ql_str
 //
 // The array lives in every device's memory from the moment the library is loaded until
 // the process exits.  In host code its name only stands in for it; the device address is
-// looked up once per device with cudaGetSymbolAddress, with that device current, on the
-// first call made on that device (so that first call should come before any stream
-// capture).  All calls on a device share the array and it keeps the contents of the last
-// call: the error word and the counters are cleared on the call's stream before each
-// launch, and two calls whose device work overlaps (e.g. on two streams) race on it.
+// looked up with cudaGetSymbolAddress, with the device current, on the first call made in
+// a device's current context (so that first call should come before any stream capture),
+// and looked up again when the context changes (after a device reset the module, and
+// with it the array, may sit at another address).  All calls on a device share the array
+// and it keeps the contents of the last call: the arrival counters are cleared on the
+// call's stream before each launch, the error word stays set until
+// qlinear_w4a16_noalloc_read_error reads it, and two calls whose device work overlaps
+// (e.g. on two streams) race on it.
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
@@ -626,20 +651,44 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes]
 
 constexpr int kMaxDevices = 64;
 
-// Device address of g_noalloc_scratch on the current device (looked up once per device).
+// The current context (cuCtxGetCurrent, looked up once through the runtime: no link
+// against libcuda).  nullptr when it cannot be queried.
+void* current_context() {
+  using Fn = CUresult (*)(CUcontext*);
+  static Fn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<Fn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!fn || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+  return ctx;
+}
+
+// Device address of g_noalloc_scratch on the current device: looked up once per device
+// and context (again whenever no context could be queried, e.g. before the runtime made
+// one current).
 cudaError_t noalloc_scratch(void** out) {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {nullptr};
+  static void* ctx_of[kMaxDevices] = {nullptr};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  void* ctx = current_context();
   std::lock_guard<std::mutex> lk(mu);
-  if (!addr[dev]) {
+  if (!addr[dev] || !ctx || ctx != ctx_of[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
     addr[dev] = p;
+    ctx_of[dev] = ctx;
   }
   *out = addr[dev];
   return cudaSuccess;
@@ -652,17 +701,29 @@ extern "C" ql_status qlinear_w4a16_noalloc(const uint16_t* x, const uint32_t* qw
                                            uint16_t* y, int M, int N, int K, int group,
                                            ql_stream_t stream) {
   if (group != kGroup) return QL_ERR_SHAPE;
-  if (!x || !qweight || !scales || !zeros || !y) return QL_ERR_NULL;
-  if (!shape_ok(M, N, K)) return QL_ERR_SHAPE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Call c{kW4, false, x, qweight, scales, zeros, nullptr, nullptr, nullptr, y, M, N, K,
+         nullptr, kNoAllocScratchBytes, st};
+  // every argument check before anything is enqueued on the stream
+  const ql_status chk = check_call(c);
+  if (chk != QL_OK) return chk;
   Plan p;
   if (make_plan(kW4, M, N, K, false, &p) != cudaSuccess) return QL_ERR_CUDA;
   if (p.ws_bytes > kNoAllocScratchBytes) return QL_ERR_WORKSPACE;  // beyond the fixed scratch
   void* scratch = nullptr;
   if (noalloc_scratch(&scratch) != cudaSuccess) return QL_ERR_CUDA;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // error word and arrival counters must start at zero (the partial sums need not)
-  if (cudaMemsetAsync(scratch, 0, p.partial_offset, st) != cudaSuccess) return QL_ERR_CUDA;
-  Call c{kW4, false, x, qweight, scales, zeros, nullptr, nullptr, nullptr, y, M, N, K,
-         scratch, kNoAllocScratchBytes, st};
+  // the arrival counters must start at zero (the partial sums need not; the error word
+  // keeps its flags until they are read)
+  if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + p.counter_offset, 0,
+                      p.partial_offset - p.counter_offset, st) != cudaSuccess)
+    return QL_ERR_CUDA;
+  c.ws = scratch;
   return run(c);
+}
+
+extern "C" ql_status qlinear_w4a16_noalloc_read_error(uint32_t* flags, ql_stream_t stream) {
+  if (!flags) return QL_ERR_NULL;
+  void* scratch = nullptr;
+  if (noalloc_scratch(&scratch) != cudaSuccess) return QL_ERR_CUDA;
+  return qlinear_read_error(scratch, flags, stream);
 }

@@ -16,7 +16,7 @@ from . import (QL_FMT_LUT4, QL_FMT_W2, QL_FMT_W3, QL_FMT_W4, QL_FMT_W8, QL_STRAT
                qlinear_debug_dequant, qlinear_policy_lookup,
                qlinear_debug_unpack, qlinear_dequant_fp16, qlinear_lut4, qlinear_pack,
                qlinear_matmul, qlinear_pack_params, qlinear_pack_params_grouped,
-               qlinear_prefill,
+               qlinear_prefill, qlinear_prefill_fused, qlinear_read_error,
                qlinear_pack_tilecoo, qlinear_w2a16, qlinear_w3a16, qlinear_w4a16,
                qlinear_w4a16_outlier,
                qlinear_w8a16, qlinear_workspace_bytes)
@@ -88,6 +88,11 @@ class QuantLinear:
                              self.workspace, stream, group=self.group)
         return y
 
+    def read_error(self, stream=None) -> int:
+        """Sticky error flags of the calls that used this layer's workspace (then cleared);
+        0 = every device wait completed."""
+        return qlinear_read_error(self.workspace, stream)
+
     def _group128(self, what: str) -> None:
         if self.group != 128:
             raise ValueError(f"{what} reads parameters packed for group 128")
@@ -118,6 +123,20 @@ class QuantLinear:
             w_fp16 = self._w_fp16
         qlinear_prefill(self.fmt, x.view(torch.int16), self.qweight, self.p0, self.p1,
                         w_fp16.view(torch.int16), y.view(torch.int16), M, self.N, self.K, stream)
+        return y
+
+    def prefill_fused(self, x: torch.Tensor, y: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+        """y[M, N] = x[M, K] . W for any M, the weights dequantized inside the tensor-core
+        GEMM (no fp16 weight matrix).  Dense part only (no outliers)."""
+        if self.tile is not None:
+            raise ValueError("prefill covers the dense formats; the outlier layer has none")
+        self._group128("prefill")
+        M = x.shape[0]
+        if y is None:
+            y = torch.empty((M, self.N), dtype=torch.float16, device=self.device)
+        qlinear_prefill_fused(self.fmt, x.view(torch.int16), self.qweight, self.p0, self.p1,
+                              y.view(torch.int16), M, self.N, self.K, stream)
         return y
 
     def matmul(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, stream=None,

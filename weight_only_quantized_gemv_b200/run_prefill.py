@@ -1,8 +1,9 @@
-"""Time the prefill path of one layer: stand-alone dequantization to fp16, the dense GEMM
-after it, and (for comparison) the fused GEMV run over 16-row slices of x.
+"""Time the prefill paths of one layer: stand-alone dequantization to fp16, the dense
+tensor-core GEMM after it, the GEMM with the dequantization fused into it, and (for
+comparison) the fused GEMV run over 16-row slices of x.
 
     python -m weight_only_quantized_gemv_b200.run_prefill --fmt w4 --K 8192 --N 28672 \
-        --M 512 [--launches 4] [--time] [--only dequant|prefill|gemv]
+        --M 512 [--launches 4] [--time] [--only dequant|prefill|fused|gemv]
 
 Packed codes and parameters are random bytes of the right sizes, and each copy has its
 own fp16 weight buffer; the copies (enough of them to exceed twice the L2 size) are
@@ -13,6 +14,7 @@ one JSON line:
 
 * dequant: algorithmic bytes = codes + parameters + the fp16 output (2 N K);
 * gemm: 2 M N K flops, its time taken as prefill minus dequant;
+* fused: 2 M N K flops over the fused kernel's time;
 * gemv: ceil(M / 16) launches of the fused GEMV (fp16 out) for the same M rows.
 """
 from __future__ import annotations
@@ -24,7 +26,8 @@ import math
 import torch
 
 from . import (FORMATS, QL_FMT_LUT4, qlinear_dequant_fp16, qlinear_lut4, qlinear_prefill,
-               qlinear_w2a16, qlinear_w4a16, qlinear_w8a16, qlinear_workspace_bytes)
+               qlinear_prefill_fused, qlinear_prefill_read_error, qlinear_w2a16,
+               qlinear_w4a16, qlinear_w8a16, qlinear_workspace_bytes)
 
 _UNIFORM = {2: qlinear_w2a16, 4: qlinear_w4a16, 8: qlinear_w8a16}
 L2_BYTES = 126 * 2 ** 20
@@ -46,7 +49,7 @@ def main() -> None:
     ap.add_argument("--launches", type=int, default=4)
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--time", action="store_true")
-    ap.add_argument("--only", choices=["dequant", "prefill", "gemv"], default=None)
+    ap.add_argument("--only", choices=["dequant", "prefill", "fused", "gemv"], default=None)
     a = ap.parse_args()
     fmt, K, N, M = FORMATS[a.fmt], a.K, a.N, a.M
     dev = torch.device("cuda:0")
@@ -80,6 +83,10 @@ def main() -> None:
         c = i % copies
         qlinear_prefill(fmt, x, q[c], p0[c], p1[c], w[c], y, M, N, K)
 
+    def fused(i):
+        c = i % copies
+        qlinear_prefill_fused(fmt, x, q[c], p0[c], p1[c], y, M, N, K)
+
     def gemv(i):
         c = i % copies
         for m0 in range(0, M, 16):
@@ -89,7 +96,7 @@ def main() -> None:
             else:
                 _UNIFORM[fmt](x[m0:], q[c], p0[c], p1[c], y[m0:], m, N, K, ws)
 
-    parts = {"dequant": dequant, "prefill": prefill, "gemv": gemv}
+    parts = {"dequant": dequant, "prefill": prefill, "fused": fused, "gemv": gemv}
     chosen = [a.only] if a.only else list(parts)
     if not a.time:
         for name in chosen:
@@ -122,8 +129,12 @@ def main() -> None:
         if "dequant" in t:
             g = t["prefill"] - t["dequant"]
             out.update(gemm_us=round(g, 2), gemm_TFLOPs=round(2 * M * N * K / g / 1e6, 1))
+    if "fused" in t:
+        out.update(fused_us=round(t["fused"], 2),
+                   fused_TFLOPs=round(2 * M * N * K / t["fused"] / 1e6, 1))
     if "gemv" in t:
         out["gemv_slices_us"] = round(t["gemv"], 2)
+    out["error_flags"] = qlinear_prefill_read_error()
     print(json.dumps(out))
 
 
