@@ -524,6 +524,11 @@ def run_gpu(args):
     # one graph holds 10 steps (60 launches), a one-step graph covers the remainder.
     g10, g1 = capture(10), capture(1)
     torch.cuda.synchronize()
+    # both graphs run once before the warm-up steps: a graph's first launch uploads it to
+    # the device, which must not land in the timed region (with few steps it would)
+    g10.replay()
+    g1.replay()
+    torch.cuda.synchronize()
 
     def steps(n):
         for _ in range(n // 10):

@@ -159,10 +159,12 @@ ql_status qlinear_read_error(void* workspace, uint32_t* flags, ql_stream_t strea
  *                       most 2^22 more rounds; 0 restores the default 2^22
  *   producer_delay_us : CTA 0's producer waits this long before its first copy
  *   consumer_hold_us  : CTA 0's first consumer warp holds its first stage this long
- *                       before releasing it (group-128 and per-channel kernels)
+ *                       before releasing it
  * Delays are at most 65535 us (QL_ERR_SHAPE otherwise); (0, 0, 0) restores normal
  * operation.  A delay shorter than the second wait gives flagged calls with correct
- * results.  Not thread-safe with respect to concurrent GEMV calls' settings. */
+ * results.  While a setting is active, the W4 kernels for M = 1 and M = 9..16 run as
+ * instances compiled with these hooks (the other kernels keep their fixed 2^22-round limit
+ * and no hooks).  Not thread-safe with respect to concurrent GEMV calls' settings. */
 ql_status qlinear_debug_wait_test(uint32_t wait_limit, uint32_t producer_delay_us,
                                   uint32_t consumer_hold_us);
 
@@ -283,11 +285,24 @@ ql_status qlinear_prefill(int fmt, const uint16_t* x, const void* packed, const 
  * weights qlinear_dequant_fp16 would write, dequantized inside the GEMM (the NF4 page's
  * codes -> FP16 -> matmul, with FP16 kept in shared memory as the tensor cores' operand
  * instead of written back).  fmt W2 / W4 / W8 (group 128) or LUT4; packed, p0, p1 as for
- * qlinear_dequant_fp16; x 16-byte aligned, y 2-byte aligned; any M >= 1, N % 16 == 0,
- * K % 128 == 0.  Asynchronous on `stream`; allocates nothing. */
+ * qlinear_dequant_fp16 but 16-byte aligned (except the LUT, 2-byte); x 16-byte aligned, y
+ * 2-byte aligned; any M >= 1, N % 16 == 0, K % 128 == 0.  Asynchronous on `stream`;
+ * allocates nothing.
+ *   workspace : NULL, or device memory of qlinear_prefill_workspace_bytes(M, N, K) bytes,
+ *               16-byte aligned and zero-filled before its first use (the kernel leaves it
+ *               zero again).  With a workspace the k-blocks of all output tiles are shared
+ *               out evenly over one CTA per SM (stream-K: tiles split between CTAs meet in
+ *               the workspace, summed in a fixed order, so results are reproducible);
+ *               without one each CTA takes whole 128 x 256 (M > 128) or 128 x 128 tiles.
+ *               QL_ERR_WORKSPACE if it is too small.  Calls sharing a workspace must not
+ *               overlap in time. */
 ql_status qlinear_prefill_fused(int fmt, const uint16_t* x, const void* packed, const void* p0,
                                 const void* p1, uint16_t* y, int M, int N, int K,
-                                ql_stream_t stream);
+                                void* workspace, size_t workspace_bytes, ql_stream_t stream);
+
+/* Bytes of the qlinear_prefill_fused workspace on the current device (0 for an unsupported
+ * shape). */
+size_t qlinear_prefill_workspace_bytes(int M, int N, int K);
 
 /* Sticky flags of the prefill GEMM kernels' bounded waits on the current device (1: a
  * pipeline stage's wait ran out, 2: an accumulator's wait ran out; results of such a call
@@ -345,7 +360,7 @@ ql_status qlinear_codebook(const uint16_t* x, const uint8_t* codes, const uint16
 
 typedef enum {
   QL_STRATEGY_GEMV = 0,    /* the fused GEMV (over 16-row slices of x when M > 16) */
-  QL_STRATEGY_PREFILL = 1  /* qlinear_prefill: dequantize to fp16, then one dense GEMM */
+  QL_STRATEGY_PREFILL = 1  /* the tensor-core prefill GEMM (qlinear_prefill / _fused) */
 } ql_strategy;
 
 typedef struct {
@@ -379,8 +394,8 @@ ql_status qlinear_policy_lookup(int fmt, int M, int N, int K, ql_policy_entry* o
  *   GEMV    : the format's GEMV entry (qlinear_w4a16 ...) on each 16-row slice of x / y in
  *             turn, all with `workspace` (at least qlinear_workspace_bytes(fmt, min(M, 16), N,
  *             K) bytes);
- *   PREFILL : qlinear_prefill into w_fp16 (N * K fp16).  When w_fp16 is NULL the GEMV is
- *             used instead.
+ *   PREFILL : qlinear_prefill into w_fp16 (N * K fp16) when w_fp16 is given, else
+ *             qlinear_prefill_fused without a workspace (whole tiles per CTA).
  * Arguments as in those entries (p0 / p1: scales / zeros, or lut16 / absmax for LUT4; group
  * 128, LUT block 64).  Returns the first non-OK status of the calls it makes. */
 ql_status qlinear_matmul(int fmt, const uint16_t* x, const void* packed, const void* p0,

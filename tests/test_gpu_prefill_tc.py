@@ -3,7 +3,9 @@ oracle on the oracle's fp16 weights.
 
 * qlinear_prefill_fused (weights dequantized inside the GEMM) for every format, on shapes
   with a ragged last 128-row tile (N % 128 != 0) and batch sizes on both sides of the token
-  tiles (128 and 256 rows of x), including a partial last token tile;
+  tiles (128 and 256 rows of x), including a partial last token tile, with the stream-K
+  schedule (tiles split between CTAs, down to one k-block per CTA on small layers) and with
+  whole tiles per CTA;
 * qlinear_prefill (stand-alone dequantization, then the same GEMM on the fp16 weights) at
   the batch sizes the older tests do not reach;
 * the same call twice (the persistent CTAs' pipeline phases carry over between tiles, not
@@ -63,6 +65,41 @@ def test_prefill_fused_parity(fmt, K, N, M):
     x = gen.activations(1900 + M, M, K)
     y = _np(lay.prefill_fused(torch.from_numpy(x).to(DEV)))
     assert_parity(y, oracle.prefill_matmul(x, w16), what=f"fused {fmt} {K}x{N} M={M}")
+
+
+@pytest.mark.parametrize("M", [1, 17, 129, 300])
+@pytest.mark.parametrize("K,N", [(384, 208), (2048, 1168)])
+@pytest.mark.parametrize("fmt", ["w2", "w4", "lut4"])
+def test_prefill_fused_whole_tiles_parity(fmt, K, N, M):
+    lay, w16 = _layer(fmt, K, N, 710)
+    x = gen.activations(1930 + M, M, K)
+    y = _np(lay.prefill_fused(torch.from_numpy(x).to(DEV), stream_k=False))
+    assert_parity(y, oracle.prefill_matmul(x, w16), what=f"whole tiles {fmt} {K}x{N} M={M}")
+
+
+def test_prefill_fused_stream_k_matches_whole_tiles():
+    """Same fp16 weights and x: the two schedules differ only in how k-blocks are summed."""
+    K, N, M = 4096, 1168, 300
+    lay, w16 = _layer("w4", K, N, 715)
+    x = torch.from_numpy(gen.activations(1940, M, K)).to(DEV)
+    a = _np(lay.prefill_fused(x, stream_k=True))
+    b = _np(lay.prefill_fused(x, stream_k=False))
+    assert_parity(a, b, what="stream-K vs whole tiles")
+    assert_parity(a, oracle.prefill_matmul(x.cpu().numpy(), w16), what="stream-K")
+
+
+def test_prefill_fused_workspace_checks():
+    K, N, M = 1024, 512, 300
+    lay, _ = _layer("w4", K, N, 716)
+    x = torch.from_numpy(gen.activations(1941, M, K)).to(DEV)
+    y = torch.empty((M, N), dtype=torch.float16, device=DEV)
+    small = torch.zeros(64, dtype=torch.int32, device=DEV)
+    with pytest.raises(ql.QLinearError) as err:
+        ql.qlinear_prefill_fused(4, x.view(torch.int16), lay.qweight, lay.p0, lay.p1,
+                                 y.view(torch.int16), M, N, K, small)
+    assert err.value.status == 5  # QL_ERR_WORKSPACE
+    assert ql.qlinear_prefill_workspace_bytes(M, N, K) > 0
+    assert ql.qlinear_prefill_workspace_bytes(M, N + 1, K) == 0
 
 
 @pytest.mark.parametrize("M", [129, 256, 300, 520])

@@ -8,7 +8,8 @@ makes one wait run out on purpose:
   * a consumer that holds its first stage for 5 ms -> the producer's wait to refill it
     runs out -> flag 2.
 The delays are far below the 2^22-round second wait, so the flagged calls still finish
-with correct results; the next call with normal settings reports no flag.
+with correct results; the next call with normal settings reports no flag.  The hooks are
+compiled into the W4 kernels for M = 1 and M = 9..16 only, which these cases use.
 """
 import os
 
@@ -50,7 +51,7 @@ def _forward(lay, xd):
     return y.float().cpu().numpy(), lay.read_error()
 
 
-@pytest.mark.parametrize("M", [1, 4])
+@pytest.mark.parametrize("M", [1, 12])
 def test_late_copy_sets_full_flag(M):
     import weight_only_quantized_gemv_b200 as ql
     lay, xd, ref = _case(3100 + M, 1024, 256, M)

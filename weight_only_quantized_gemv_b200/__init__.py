@@ -78,7 +78,8 @@ _SIGS = {
     "qlinear_w4a16_noalloc_read_error": (_I, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "qlinear_dequant_fp16": (_I, [_I, _P, _P, _P, _P, _I, _I, _P]),
     "qlinear_prefill": (_I, [_I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
-    "qlinear_prefill_fused": (_I, [_I, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "qlinear_prefill_fused": (_I, [_I, _P, _P, _P, _P, _P, _I, _I, _I, _P, _SZ, _P]),
+    "qlinear_prefill_workspace_bytes": (_SZ, [_I, _I, _I]),
     "qlinear_prefill_read_error": (_I, [ctypes.POINTER(ctypes.c_uint32), _P]),
     "qlinear_policy_set": (_I, [ctypes.POINTER(ql_policy_entry), _I]),
     "qlinear_policy_size": (_I, []),
@@ -307,11 +308,19 @@ def qlinear_prefill(fmt, x, packed, p0, p1, w_fp16, y, M, N, K, stream=None):
     return y
 
 
-def qlinear_prefill_fused(fmt, x, packed, p0, p1, y, M, N, K, stream=None):
-    """``y[M, N] = x[M, K] @ W^T`` with the weights dequantized inside the tensor-core GEMM."""
+def qlinear_prefill_fused(fmt, x, packed, p0, p1, y, M, N, K, workspace=None, stream=None):
+    """``y[M, N] = x[M, K] @ W^T`` with the weights dequantized inside the tensor-core GEMM;
+    with a (zero-filled) workspace the k-blocks are shared out over the SMs (stream-K)."""
     _check(_lib.qlinear_prefill_fused(fmt, _ptr(x), _ptr(packed), _ptr(p0), _ptr(p1), _ptr(y),
-                                      M, N, K, _stream(stream)), "qlinear_prefill_fused")
+                                      M, N, K, _ptr(workspace),
+                                      workspace.numel() * workspace.element_size()
+                                      if workspace is not None else 0, _stream(stream)),
+           "qlinear_prefill_fused")
     return y
+
+
+def qlinear_prefill_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_lib.qlinear_prefill_workspace_bytes(M, N, K))
 
 
 def qlinear_prefill_read_error(stream=None) -> int:

@@ -37,10 +37,10 @@
 //  * The outlier variant adds the Tile-COO entries of each unit into a shared fp32
 //    y tile, reading x from the same stage the dense path uses; the y tile joins
 //    the dense sums at the end of the unit range, before the split-K fix-up.
-//  * Every mbarrier wait is bounded.  A wait that passes its limit sets a bit in the
-//    workspace error word, then waits at most as long again for the late copy (or the
-//    late release) and carries on; a lost copy can corrupt results but never hang the
-//    GPU, and every copy a CTA issued has landed when it exits unless a wait gave up.
+//  * Every mbarrier wait is bounded.  A wait that runs out sets a bit in the workspace
+//    error word and carries on, so a lost copy can corrupt results but never hang the
+//    GPU.  Instances built for tests of the waits (TH) can shorten the limit, delay a
+//    copy or hold a stage, and wait once more after flagging.
 #pragma once
 #include <cuda.h>  // CUtensorMap
 #include <cuda_fp16.h>
@@ -217,14 +217,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_
   return false;
 }
 
-// Wait for a stage's phase.  Past P.wait_limit rounds the wait sets `bit` in the error
-// word and goes on waiting for at most kSpinLimit more rounds (a late copy still lands
-// before it is read); if it then gives up too, the results are undefined.
+// Wait for a stage's phase, bounded by kSpinLimit rounds; a wait that gives up sets `bit` in
+// the error word and carries on (the results are then undefined).  TH: the instances built
+// for tests of the bounded waits, where the limit is P.wait_limit and a wait that passes it
+// sets the flag and then waits at most kSpinLimit more rounds, so that a late copy still
+// lands before it is read.  (Kept out of the other instances: in the unit loop the longer
+// form costs the single-row kernel about 6 %.)
+template <bool TH>
 __device__ __forceinline__ void stage_wait(const GemvParams& P, uint32_t bar, uint32_t parity,
                                            uint32_t bit) {
-  if (!mbar_wait(bar, parity, P.wait_limit)) {
-    atomicOr(P.err, bit);
-    mbar_wait(bar, parity, kSpinLimit);
+  if constexpr (TH) {
+    if (!mbar_wait(bar, parity, P.wait_limit)) {
+      atomicOr(P.err, bit);
+      mbar_wait(bar, parity, kSpinLimit);
+    }
+  } else {
+    if (!mbar_wait(bar, parity, kSpinLimit)) atomicOr(P.err, bit);
   }
 }
 
@@ -403,7 +411,8 @@ __host__ __device__ __forceinline__ int cta_of_unit(int u, int U, int C) {
 
 // ---------------------------------------------------------------------------
 
-template <int FMT, int MT, bool OUTL, int WPU_, bool M1_ = false, int OCC_ = 0, int NS_ = 1>
+template <int FMT, int MT, bool OUTL, int WPU_, bool M1_ = false, int OCC_ = 0, int NS_ = 1,
+          bool TH = false>
 struct Gemv {
   using C_ = Cfg<FMT, MT, OUTL, WPU_, M1_, OCC_, NS_>;
   static constexpr int NS = C_::NS;
@@ -662,7 +671,7 @@ struct Gemv {
       for (int e = 0; e < NACC; ++e)
         if (!kLut) v[i][e] *= (e & 2) ? kTwo24 * Fmt<FMT>::kHiScale : kTwo24;
     }
-    if constexpr (OUTL) {
+    if constexpr (OUTL) {  // the outlier sums of this warp's tiles, then cleared
       const int gi = lane >> 2, t4 = lane & 3;
 #pragma unroll
       for (int i = 0; i < T; ++i) {
@@ -678,6 +687,9 @@ struct Gemv {
           }
         }
       }
+      // the next run's units add into the tile only after every warp has read and cleared
+      // its part (a warp that went on early would add into sums another warp still reads)
+      consumer_sync(NC * 32);
     }
     if (warp * T >= tb) return;
     if (whole) {
@@ -797,7 +809,9 @@ struct Gemv {
             : "memory");
       }
     };
-    if ((P.test_us & 0xFFFFu) && blockIdx.x == 0) test_delay(P.test_us & 0xFFFFu);
+    if constexpr (TH) {  // tests of the bounded waits: CTA 0's first copy comes late
+      if ((P.test_us & 0xFFFFu) && blockIdx.x == 0) test_delay(P.test_us & 0xFFFFu);
+    }
     const int b0 = u0 / P.G, g0 = u0 - b0 * P.G;
     int b = b0, g = g0;
     const int pre = n < S ? n : S;
@@ -813,7 +827,7 @@ struct Gemv {
     g = g0;
     for (int i = 0; i < n; ++i) {
       if (i >= S) {
-        stage_wait(P, bars + 8 * (S + i % S), ((i / S) - 1) & 1, kErrEmptyTimeout);
+        stage_wait<TH>(P, bars + 8 * (S + i % S), ((i / S) - 1) & 1, kErrEmptyTimeout);
         weights(i, b, g);
       }
       activations(i, g);
@@ -842,7 +856,7 @@ struct Gemv {
     const int s = i % S;
     const int tb = tiles_in_block(b, P.ntiles);
     const uint32_t st = ring + s * C_::kStageBytes;
-    stage_wait(P, bars + 8 * s, (i / S) & 1, kErrFullTimeout);
+    stage_wait<TH>(P, bars + 8 * s, (i / S) & 1, kErrFullTimeout);
     uint4 xr[4], xr2[4];
     read_x(P, st, lane, xr, xr2);
     if constexpr (OUTL) {
@@ -1023,7 +1037,7 @@ struct Gemv {
     const int s = i % S;
     const int tb = tiles_in_block(b, P.ntiles);
     const uint32_t st = ring + s * C_::kStageBytes;
-    stage_wait(P, bars + 8 * s, (i / S) & 1, kErrFullTimeout);
+    stage_wait<TH>(P, bars + 8 * s, (i / S) & 1, kErrFullTimeout);
     uint4 xr[4], xr2[4];
     read_x(P, st, lane, xr, xr2);
     const int t0 = kTW * sub;
@@ -1096,9 +1110,11 @@ struct Gemv {
     uint32_t orc[3] = {0, 0, 0}, oval[3] = {0, 0, 0};
     // tests of the bounded waits: CTA 0's warp 0 takes stage 0 and holds it for a while
     // before its first unit releases it (waiting for a completed phase again returns at once)
-    if ((P.test_us >> 16) && blockIdx.x == 0 && warp == 0 && n > 0) {
-      stage_wait(P, smem_addr(smem) + C_::kBarOff, 0, kErrFullTimeout);
-      test_delay(P.test_us >> 16);
+    if constexpr (TH) {
+      if ((P.test_us >> 16) && blockIdx.x == 0 && warp == 0 && n > 0) {
+        stage_wait<TH>(P, smem_addr(smem) + C_::kBarOff, 0, kErrFullTimeout);
+        test_delay(P.test_us >> 16);
+      }
     }
     if constexpr (OUTL) {
       consumer_sync(NC * 32);  // the Tile-COO offsets are in shared memory
@@ -1127,13 +1143,13 @@ struct NoXMap {
 template <bool XT> struct XMapParam { using type = NoXMap; };
 template <> struct XMapParam<true> { using type = CUtensorMap; };
 
-template <int FMT, int MT, bool OUTL, int WPU, bool M1, int OCC, int NS = 1>
+template <int FMT, int MT, bool OUTL, int WPU, bool M1, int OCC, int NS = 1, bool TH = false>
 __global__ void __launch_bounds__(Cfg<FMT, MT, OUTL, WPU, M1, OCC, NS>::kThreads,
                                   Cfg<FMT, MT, OUTL, WPU, M1, OCC, NS>::kMinCtas)
     qgemv_kernel(const GemvParams P, const __grid_constant__ typename XMapParam<!M1>::type xm) {
   const CUtensorMap* xmap = nullptr;
   if constexpr (!M1) xmap = &xm;
-  using G_ = Gemv<FMT, MT, OUTL, WPU, M1, OCC, NS>;
+  using G_ = Gemv<FMT, MT, OUTL, WPU, M1, OCC, NS, TH>;
   using C_ = Cfg<FMT, MT, OUTL, WPU, M1, OCC, NS>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

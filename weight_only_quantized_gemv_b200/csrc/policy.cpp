@@ -103,8 +103,12 @@ extern "C" ql_status qlinear_matmul(int fmt, const uint16_t* x, const void* pack
   if (!fmt_ok(fmt)) return QL_ERR_UNSUPPORTED;
   if (M < 1) return QL_ERR_SHAPE;
   const qpolicy::Choice c = qpolicy::lookup(fmt, false, M, N, K);
-  if (c.strategy == QL_STRATEGY_PREFILL && w_fp16)
-    return qlinear_prefill(fmt, x, packed, p0, p1, w_fp16, y, M, N, K, stream);
+  if (c.strategy == QL_STRATEGY_PREFILL) {
+    if (w_fp16) return qlinear_prefill(fmt, x, packed, p0, p1, w_fp16, y, M, N, K, stream);
+    // the tensor-core GEMM with the dequantization fused in, whole tiles per CTA (the GEMV
+    // workspace is not the stream-K workspace)
+    return qlinear_prefill_fused(fmt, x, packed, p0, p1, y, M, N, K, nullptr, 0, stream);
+  }
   // the fused GEMV, over 16-row slices of x and y
   if (!x || !y) return QL_ERR_NULL;
   for (int m0 = 0; m0 < M; m0 += 16) {

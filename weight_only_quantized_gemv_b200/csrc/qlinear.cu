@@ -48,12 +48,29 @@ struct KernelInfo {
 };
 
 template <int FMT, int MT, bool OUTL, int WPU = qlk::default_wpu(FMT, MT), bool M1 = false,
-          int OCC = 0, int NS = 1>
+          int OCC = 0, int NS = 1, bool TH = false>
 KernelInfo kernel_info() {
   using C = qlk::Cfg<FMT, MT, OUTL, WPU, M1, OCC, NS>;
   return KernelInfo{
-      reinterpret_cast<const void*>(qlk::qgemv_kernel<FMT, MT, OUTL, WPU, M1, OCC, NS>),
+      reinterpret_cast<const void*>(qlk::qgemv_kernel<FMT, MT, OUTL, WPU, M1, OCC, NS, TH>),
       C::kThreads, C::kSmemBytes, C::NC, C::T, !M1};
+}
+
+// Instances with the test hooks of the bounded waits (same shared memory and threads as the
+// instance they stand in for): W4 with one row of x (three and two CTAs per SM) and W4 at
+// M = 9..16.  Other kernels run without the hooks.
+bool test_kernel(int fmt, int MT, bool outl, int wpu, bool m1, bool occ2, int ns, KernelInfo* k) {
+  if (fmt != kW4 || outl || ns != 1) return false;
+  if (MT == 2) {
+    *k = kernel_info<kW4, 2, false, 2, false, 0, 1, true>();
+    return true;
+  }
+  if (m1 && wpu == 1) {
+    *k = occ2 ? kernel_info<kW4, 1, false, 1, true, 2, 1, true>()
+              : kernel_info<kW4, 1, false, 1, true, 0, 1, true>();
+    return true;
+  }
+  return false;
 }
 
 // Finer quantization groups (NS sub-groups per 128-k unit): two warps per unit for every
@@ -358,7 +375,16 @@ ql_status run(const Call& c) {
   P.C = p.C;
   P.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
   P.test_us = g_test_us.load(std::memory_order_relaxed);
-  const KernelInfo k = select_kernel(c.fmt, p.MT, c.outl, p.WPU, p.M1, p.OCC2, p.NS);
+  KernelInfo k = select_kernel(c.fmt, p.MT, c.outl, p.WPU, p.M1, p.OCC2, p.NS);
+  if (P.wait_limit != qlk::kSpinLimit || P.test_us != 0) {  // qlinear_debug_wait_test is active
+    KernelInfo kt;
+    if (test_kernel(c.fmt, p.MT, c.outl, p.WPU, p.M1, p.OCC2, p.NS, &kt)) {
+      int dev = 0, occ = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess || prepare_kernel(kt, dev, &occ) != cudaSuccess)
+        return QL_ERR_CUDA;
+      k = kt;
+    }
+  }
   // Programmatic stream serialization: the kernel may start while the previous kernel in
   // the stream drains; it requests only static weight bytes before griddepcontrol.wait.
   cudaLaunchConfig_t cfg = {};

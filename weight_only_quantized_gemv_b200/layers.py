@@ -12,11 +12,12 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (QL_FMT_LUT4, QL_FMT_W2, QL_FMT_W3, QL_FMT_W4, QL_FMT_W8, QL_STRATEGY_PREFILL,
-               qlinear_debug_dequant, qlinear_policy_lookup,
+from . import (QL_FMT_LUT4, QL_FMT_W2, QL_FMT_W3, QL_FMT_W4, QL_FMT_W8,
+               qlinear_debug_dequant,
                qlinear_debug_unpack, qlinear_dequant_fp16, qlinear_lut4, qlinear_pack,
                qlinear_matmul, qlinear_pack_params, qlinear_pack_params_grouped,
-               qlinear_prefill, qlinear_prefill_fused, qlinear_read_error,
+               qlinear_prefill, qlinear_prefill_fused, qlinear_prefill_workspace_bytes,
+               qlinear_read_error,
                qlinear_pack_tilecoo, qlinear_w2a16, qlinear_w3a16, qlinear_w4a16,
                qlinear_w4a16_outlier,
                qlinear_w8a16, qlinear_workspace_bytes)
@@ -126,39 +127,43 @@ class QuantLinear:
         return y
 
     def prefill_fused(self, x: torch.Tensor, y: Optional[torch.Tensor] = None,
-                      stream=None) -> torch.Tensor:
+                      stream=None, stream_k: bool = True) -> torch.Tensor:
         """y[M, N] = x[M, K] . W for any M, the weights dequantized inside the tensor-core
-        GEMM (no fp16 weight matrix).  Dense part only (no outliers)."""
+        GEMM (no fp16 weight matrix); stream_k shares the k-blocks out over the SMs through a
+        workspace the layer keeps.  Dense part only (no outliers)."""
         if self.tile is not None:
             raise ValueError("prefill covers the dense formats; the outlier layer has none")
         self._group128("prefill")
         M = x.shape[0]
         if y is None:
             y = torch.empty((M, self.N), dtype=torch.float16, device=self.device)
+        ws = self._prefill_workspace(M) if stream_k else None
         qlinear_prefill_fused(self.fmt, x.view(torch.int16), self.qweight, self.p0, self.p1,
-                              y.view(torch.int16), M, self.N, self.K, stream)
+                              y.view(torch.int16), M, self.N, self.K, ws, stream)
         return y
 
-    def matmul(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, stream=None,
-               allow_prefill: bool = True) -> torch.Tensor:
+    def _prefill_workspace(self, M: int) -> torch.Tensor:
+        """The zero-filled stream-K workspace of the fused prefill, grown as M needs."""
+        need = qlinear_prefill_workspace_bytes(M, self.N, self.K)
+        ws = getattr(self, "_pf_ws", None)
+        if ws is None or ws.numel() * 4 < need:
+            ws = torch.zeros(need // 4 + 64, dtype=torch.int32, device=self.device)
+            self._pf_ws = ws
+        return ws
+
+    def matmul(self, x: torch.Tensor, y: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
         """y[M, N] = x[M, K] . W for any M, dispatched by the library's policy map (the fused
-        GEMV, over 16-row slices when M > 16, or the prefill path).  The layer's fp16 weight
-        buffer for prefill is allocated on the first call the policy sends to prefill."""
+        GEMV, over 16-row slices when M > 16, or the tensor-core prefill GEMM with the
+        dequantization fused in)."""
         if self.tile is not None:
             raise ValueError("the policy map covers the dense formats")
         self._group128("matmul")
         M = x.shape[0]
         if y is None:
             y = torch.empty((M, self.N), dtype=torch.float16, device=self.device)
-        wbuf = None
-        decision, _ = qlinear_policy_lookup(self.fmt, M, self.N, self.K)
-        if allow_prefill and decision["strategy"] == QL_STRATEGY_PREFILL:
-            if getattr(self, "_w_fp16", None) is None:
-                self._w_fp16 = torch.empty((self.N, self.K), dtype=torch.float16,
-                                           device=self.device)
-            wbuf = self._w_fp16.view(torch.int16)
         qlinear_matmul(self.fmt, x.view(torch.int16), self.qweight, self.p0, self.p1,
-                       y.view(torch.int16), M, self.N, self.K, self.workspace, wbuf, stream)
+                       y.view(torch.int16), M, self.N, self.K, self.workspace, None, stream)
         return y
 
     def debug_unpack(self, stream=None) -> torch.Tensor:

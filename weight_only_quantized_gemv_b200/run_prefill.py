@@ -26,7 +26,8 @@ import math
 import torch
 
 from . import (FORMATS, QL_FMT_LUT4, qlinear_dequant_fp16, qlinear_lut4, qlinear_prefill,
-               qlinear_prefill_fused, qlinear_prefill_read_error, qlinear_w2a16,
+               qlinear_prefill_fused, qlinear_prefill_read_error,
+               qlinear_prefill_workspace_bytes, qlinear_w2a16,
                qlinear_w4a16, qlinear_w8a16, qlinear_workspace_bytes)
 
 _UNIFORM = {2: qlinear_w2a16, 4: qlinear_w4a16, 8: qlinear_w8a16}
@@ -50,6 +51,7 @@ def main() -> None:
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--time", action="store_true")
     ap.add_argument("--only", choices=["dequant", "prefill", "fused", "gemv"], default=None)
+    ap.add_argument("--stream-k", type=int, default=1, help="fused: 1 = stream-K, 0 = whole tiles")
     a = ap.parse_args()
     fmt, K, N, M = FORMATS[a.fmt], a.K, a.N, a.M
     dev = torch.device("cuda:0")
@@ -83,9 +85,12 @@ def main() -> None:
         c = i % copies
         qlinear_prefill(fmt, x, q[c], p0[c], p1[c], w[c], y, M, N, K)
 
+    pf_ws = torch.zeros(qlinear_prefill_workspace_bytes(M, N, K) // 4 + 64, dtype=torch.int32,
+                        device=dev) if a.stream_k else None
+
     def fused(i):
         c = i % copies
-        qlinear_prefill_fused(fmt, x, q[c], p0[c], p1[c], y, M, N, K)
+        qlinear_prefill_fused(fmt, x, q[c], p0[c], p1[c], y, M, N, K, pf_ws)
 
     def gemv(i):
         c = i % copies

@@ -130,7 +130,6 @@ def tune_layer(fmt: int, K: int, N: int, m_list: Sequence[int], reps: int, log,
               for _ in range(copies)]
         p1 = [torch.randint(0, 1 << bits, (G * N,), device=dev, generator=gen).half()
               .view(torch.int16) for _ in range(copies)]
-    wbuf = [torch.empty(N * K, dtype=torch.int16, device=dev) for _ in range(copies)]
     Mmax = max(m_list)
     x = torch.randn(Mmax, K, device=dev, generator=gen).half().view(torch.int16)
     y = torch.empty(Mmax, N, device=dev, dtype=torch.int16)
@@ -146,7 +145,7 @@ def tune_layer(fmt: int, K: int, N: int, m_list: Sequence[int], reps: int, log,
 
         def call(i):
             j = i % copies
-            qlinear_matmul(fmt, x, q[j], p0[j], p1[j], y, M, N, K, ws, wbuf[j])
+            qlinear_matmul(fmt, x, q[j], p0[j], p1[j], y, M, N, K, ws, None)
 
         for i in range(2 * copies):
             call(i)
@@ -203,7 +202,7 @@ def tune_layer(fmt: int, K: int, N: int, m_list: Sequence[int], reps: int, log,
         if reverted:
             entries = build_entries(fmt, N, K, best)
     qlinear_policy_set([])
-    del q, p0, p1, wbuf, x, y, ws_cache
+    del q, p0, p1, x, y, ws_cache
     torch.cuda.empty_cache()
     return entries, timings, checks
 
