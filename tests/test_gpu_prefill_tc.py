@@ -10,8 +10,12 @@ oracle on the oracle's fp16 weights.
   the batch sizes the older tests do not reach;
 * the same call twice (the persistent CTAs' pipeline phases carry over between tiles, not
   between calls), and the kernels' wait flags read back as 0;
+* forty calls on a layer whose CTAs each run 64 k-blocks, all bit-identical;
 * one-hot rows of x: y equals the fp16 weight column bit for bit (a single exact product);
-* the target layer (8192 x 28672, W4) at M = 512 on sampled columns.
+* the target layer (8192 x 28672, W4) at M = 512 on sampled columns;
+* both tile forms: one CTA per 128-row tile, and a cluster pair of CTAs per 256-row tile
+  (tcgen05 cta_group::2; QLINEAR_TC_PAIR selects), including layers whose last pair has
+  no rows for its second CTA (N / 128 odd).
 """
 import functools
 
@@ -41,6 +45,12 @@ def _cuda():
     assert ql.qlinear_prefill_read_error() == 0, "a prefill kernel wait ran out"
 
 
+@pytest.fixture(params=["pair", "single"])
+def tile_form(request, monkeypatch):
+    monkeypatch.setenv("QLINEAR_TC_PAIR", "1" if request.param == "pair" else "0")
+    return request.param
+
+
 def _layer(fmt, K, N, seed):
     if fmt == "lut4":
         lt = lut4_layer(seed, K, N)
@@ -58,9 +68,9 @@ def _np(t):
 
 
 @pytest.mark.parametrize("M", [1, 16, 17, 128, 129, 256, 300])
-@pytest.mark.parametrize("K,N", [(384, 208), (1024, 512), (2048, 1168)])
+@pytest.mark.parametrize("K,N", [(384, 208), (1024, 384), (1024, 512), (2048, 1168)])
 @pytest.mark.parametrize("fmt", ["w2", "w4", "w8", "lut4"])
-def test_prefill_fused_parity(fmt, K, N, M):
+def test_prefill_fused_parity(fmt, K, N, M, tile_form):
     lay, w16 = _layer(fmt, K, N, 700)
     x = gen.activations(1900 + M, M, K)
     y = _np(lay.prefill_fused(torch.from_numpy(x).to(DEV)))
@@ -68,16 +78,16 @@ def test_prefill_fused_parity(fmt, K, N, M):
 
 
 @pytest.mark.parametrize("M", [1, 17, 129, 300])
-@pytest.mark.parametrize("K,N", [(384, 208), (2048, 1168)])
+@pytest.mark.parametrize("K,N", [(384, 208), (1024, 384), (2048, 1168)])
 @pytest.mark.parametrize("fmt", ["w2", "w4", "lut4"])
-def test_prefill_fused_whole_tiles_parity(fmt, K, N, M):
+def test_prefill_fused_whole_tiles_parity(fmt, K, N, M, tile_form):
     lay, w16 = _layer(fmt, K, N, 710)
     x = gen.activations(1930 + M, M, K)
     y = _np(lay.prefill_fused(torch.from_numpy(x).to(DEV), stream_k=False))
     assert_parity(y, oracle.prefill_matmul(x, w16), what=f"whole tiles {fmt} {K}x{N} M={M}")
 
 
-def test_prefill_fused_stream_k_matches_whole_tiles():
+def test_prefill_fused_stream_k_matches_whole_tiles(tile_form):
     """Same fp16 weights and x: the two schedules differ only in how k-blocks are summed."""
     K, N, M = 4096, 1168, 300
     lay, w16 = _layer("w4", K, N, 715)
@@ -103,9 +113,10 @@ def test_prefill_fused_workspace_checks():
 
 
 @pytest.mark.parametrize("M", [129, 256, 300, 520])
+@pytest.mark.parametrize("N", [1168, 384])
 @pytest.mark.parametrize("fmt", ["w4", "lut4"])
-def test_prefill_dense_tc_parity(fmt, M):
-    K, N = 1024, 1168
+def test_prefill_dense_tc_parity(fmt, N, M, tile_form):
+    K = 1024
     lay, w16 = _layer(fmt, K, N, 720)
     x = gen.activations(1950 + M, M, K)
     wbuf = torch.empty((N, K), dtype=torch.float16, device=DEV)
@@ -115,7 +126,7 @@ def test_prefill_dense_tc_parity(fmt, M):
     assert_parity(y, oracle.prefill_matmul(x, w16), what=f"dense tc {fmt} M={M}")
 
 
-def test_prefill_fused_repeat_and_explicit_stream():
+def test_prefill_fused_repeat_and_explicit_stream(tile_form):
     K, N, M = 2048, 1168, 300
     lay, w16 = _layer("w4", K, N, 730)
     x = torch.from_numpy(gen.activations(1990, M, K)).to(DEV)
@@ -132,8 +143,31 @@ def test_prefill_fused_repeat_and_explicit_stream():
                   oracle.prefill_matmul(x.cpu().numpy(), w16), what="repeat")
 
 
+@pytest.mark.parametrize("stream_k", [False, True])
+@pytest.mark.parametrize("fmt", ["w2", "w4"])
+def test_prefill_fused_repeat_many(fmt, stream_k, tile_form):
+    """Long per-CTA runs (whole tiles: 64 k-blocks per CTA, so every ring wraps many times),
+    repeated: each result bit-identical to the first, the first within tolerance.  A shared-
+    memory slot released too early shows up here as results that differ between calls."""
+    K, N, M = 4096, 1168, 300
+    lay, w16 = _layer(fmt, K, N, 760)
+    x = torch.from_numpy(gen.activations(1995, M, K)).to(DEV)
+    y = torch.empty((M, N), dtype=torch.float16, device=DEV)
+    first = None
+    for _ in range(40):
+        lay.prefill_fused(x, y, stream_k=stream_k)
+        torch.cuda.synchronize()
+        h = y.view(torch.int16).cpu().numpy()
+        if first is None:
+            first = h.copy()
+            assert_parity(h.view(np.float16).astype(np.float64),
+                          oracle.prefill_matmul(x.cpu().numpy(), w16), what=f"repeat {fmt}")
+        else:
+            assert np.array_equal(h, first)
+
+
 @pytest.mark.parametrize("fmt", ["w4", "w8", "lut4"])
-def test_prefill_fused_one_hot_bit_exact(fmt):
+def test_prefill_fused_one_hot_bit_exact(fmt, tile_form):
     K, N = 1024, 400
     lay, w16 = _layer(fmt, K, N, 740)
     ks = [0, 5, 63, 64, 127, 128, 511, 1023]
@@ -153,7 +187,7 @@ def _big():
 
 
 @pytest.mark.slow
-def test_prefill_fused_full_size_sampled():
+def test_prefill_fused_full_size_sampled(tile_form):
     u = _big()
     K, N, M = u.K, u.N, 512
     rs = np.random.default_rng(7)

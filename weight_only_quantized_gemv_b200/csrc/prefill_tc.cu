@@ -37,6 +37,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cstdlib>
 #include <mutex>
 #include <unordered_map>
 
@@ -56,11 +57,17 @@ constexpr uint32_t kErrStage = 1u, kErrAcc = 2u;
 
 __device__ uint32_t g_tc_err;  // sticky wait-timeout flags of the prefill kernels
 
-template <int BN, bool FUSED, int FMT = kW4>
+template <int BN, bool FUSED, int FMT = kW4, bool PAIR = false>
 struct TcCfg {
   static_assert(BN == 128 || BN == 256, "token tile");
+  // PAIR: a cluster of two CTAs on two SMs computes one tile of 2 x 128 weight rows with
+  // tcgen05.mma.cta_group::2: each CTA holds its 128 rows of A and half of the tile's rows
+  // of x in its own shared memory, and its 128 rows of the accumulator in its tensor memory.
+  static constexpr int kCtas = PAIR ? 2 : 1;
+  static constexpr int kRows = kBM * kCtas;                  // weight rows per tile (MMA M)
+  static constexpr int kBRows = BN / kCtas;                  // rows of x one CTA copies
   static constexpr int kABytes = kBM * kBK * 2;              // 16 KB
-  static constexpr int kBBytes = BN * kBK * 2;               // 32 / 16 KB
+  static constexpr int kBBytes = kBRows * kBK * 2;           // 8 .. 32 KB
   // FUSED: the stage's packed codes, as bulk-copied: per 16-row tile the half chunk of the
   // stage's 64 k (W4, LUT4: quad h, 512 B; W8: quads 2h, 2h + 1, 1 KB; W2: the whole 512-B
   // chunk, whose halves interleave per lane), then the block's parameters for the group
@@ -69,24 +76,43 @@ struct TcCfg {
   static constexpr int kCodeBytes = FUSED ? 8 * kCodeChunk : 0;
   static constexpr int kParChunk = FMT == kLUT4 ? 128 : 32;  // per tile, per array
   static constexpr int kParBytes = FUSED ? (FMT == kLUT4 ? 8 * 128 : 2 * 8 * 32) : 0;
-  static constexpr int kCodeOff = kABytes + kBBytes;
-  static constexpr int kParOff = kCodeOff + kCodeBytes;
-  static constexpr int kStageBytes = (kParOff + kParBytes + 1023) / 1024 * 1024;
-  static constexpr int S0 = (232448 - 2048) / kStageBytes;   // stages that fit
-  static constexpr int S = S0 < 6 ? S0 : 6;
-  static_assert(S >= 3, "pipeline depth");
+  // A and B of one stage; FUSED: the codes and parameters of a stage live in a ring of their
+  // own (SC slots), which a producer warp fills ahead of the A / B ring: a code slot is free
+  // again as soon as the dequantizing warps have read it, long before the MMAs are done
+  // with the stage, so the codes' HBM latency is covered by SC stages instead of S
+  static constexpr int kStageBytes = kABytes + kBBytes;      // multiple of 1024
+  static constexpr int kCodeSlot = (kCodeBytes + kParBytes + 127) / 128 * 128;
+  static constexpr int kParOff = kCodeBytes;                 // inside a code slot
+  static constexpr int kBudget = 232448 - 2048;              // bytes for the two rings
+  // stages: as many as fit up to 8; FUSED: the most (up to 6) that leave six code slots
+  static constexpr int pick_s() {
+    if (!FUSED) return kBudget / kStageBytes < 8 ? kBudget / kStageBytes : 8;
+    for (int st = 6; st >= 3; --st)
+      if (kBudget - st * kStageBytes >= 6 * kCodeSlot) return st;
+    return 2;
+  }
+  static constexpr int S = pick_s();
+  static constexpr int SC0 = FUSED ? (kBudget - S * kStageBytes) / kCodeSlot : 0;
+  static constexpr int SC = SC0 < 8 ? SC0 : 8;
+  static constexpr int kCodeRingOff = S * kStageBytes;
+  static_assert(S >= 3 && (!FUSED || SC >= 6), "pipeline depth");
   static constexpr int kEpiWarp0 = 2, kEpiWarps = 4;
   static constexpr int kDqWarp0 = kEpiWarp0 + kEpiWarps;
-  static constexpr int kWarps = kDqWarp0 + (FUSED ? kDqWarps : 0);
+  static constexpr int kCodeWarp = kDqWarp0 + kDqWarps;      // FUSED: the code producer
+  static constexpr int kWarps = FUSED ? kCodeWarp + 1 : kDqWarp0;
   static constexpr int kThreads = 32 * kWarps;
-  static constexpr int kBarOff = S * kStageBytes;
-  // full[S] empty[S] accf[2] acce[2] fin cfull[S]
-  static constexpr int kSlotOff = kBarOff + 8 * (3 * S + 5);  // tensor-memory base, abort flag
+  static constexpr int kBarOff = kCodeRingOff + SC * kCodeSlot;
+  // full[S] empty[S] accf[2] acce[2] fin cfull[SC] cempty[SC]
+  static constexpr int kSlotOff = kBarOff + 8 * (2 * S + 5 + 2 * SC);  // tmem base, abort flag
   static constexpr int kSmemBytes = kSlotOff + 16 + 1024;    // + slack to align the ring
   static constexpr uint32_t kTmemCols = 2 * BN;
-  // full[s] completes on the TMA bytes of x (and W) plus one arrival per dequantizing warp;
-  // cfull[s] (FUSED) on the bytes of the stage's codes and parameters
-  static constexpr uint32_t kFullCount = 1 + (FUSED ? kDqWarps : 0);
+  // full[s] (the leader CTA's, for both CTAs of a pair) completes on the TMA bytes of x (and
+  // W) of every CTA of the tile plus one arrival per dequantizing warp; cfull[s] (FUSED, each
+  // CTA its own) on the bytes of the stage's codes and parameters
+  static constexpr uint32_t kFullCount = 1 + (FUSED ? kCtas * kDqWarps : 0);
+  static constexpr uint32_t kFullBytes = kCtas * (kBBytes + (FUSED ? 0 : kABytes));
+  static constexpr uint32_t kAccEmptyCount = kCtas * kEpiWarps;  // acce[a], the leader's
+  static_assert(kSmemBytes + 64 <= 232448, "shared memory");
 };
 
 struct TcParams {
@@ -95,8 +121,9 @@ struct TcParams {
   const void* p1;        // FUSED: packed zeros | packed absmax
   __half* y;             // [M][N]
   float* partials;       // stream-K: fp32 partial tiles, two slots per CTA (null: whole tiles)
-  uint32_t* counters;    // stream-K: arrivals per (tile, epilogue warp)
+  uint32_t* counters;    // stream-K: arrivals per (tile, CTA of the tile, epilogue warp)
   int M, N, K, G, ntiles, mtiles, tiles;
+  bool pair;             // host: launch the cluster-pair instance
 };
 
 // The k-block work of a CTA as a sequence of segments (tile t, k-blocks [kb0, kb1)).
@@ -104,13 +131,17 @@ struct TcParams {
 //  * stream-K: the flattened (tile, k-block) units [c U / C, (c + 1) U / C), U = tiles x KB,
 //    cut at tile boundaries: only a CTA's first and last segments can be partial tiles,
 //    and every CTA gets the same number of k-blocks to within one.
+// A worker is a CTA, or a cluster pair of CTAs (both follow the same sequence).
 struct SegIter {
   long long u, u1;  // stream-K: next unit, end of the range
-  int j;            // whole tiles: next tile of this CTA
-  __device__ void init(const TcParams& P, int KB) {
-    const long long U = (long long)P.tiles * KB, C = gridDim.x;
-    u = blockIdx.x * U / C;
-    u1 = (blockIdx.x + 1) * U / C;
+  int j;            // whole tiles: next tile of this worker
+  int w, W;         // this worker, number of workers
+  __device__ void init(const TcParams& P, int KB, int w_, int W_) {
+    w = w_;
+    W = W_;
+    const long long U = (long long)P.tiles * KB;
+    u = w * U / W;
+    u1 = (w + 1) * U / W;
     j = 0;
   }
   __device__ bool next(const TcParams& P, int KB, int& t, int& kb0, int& kb1) {
@@ -122,7 +153,7 @@ struct SegIter {
       u += kb1 - kb0;
       return true;
     }
-    t = blockIdx.x + j * gridDim.x;
+    t = w + j * W;
     if (t >= P.tiles) return false;
     ++j;
     kb0 = 0;
@@ -140,15 +171,30 @@ __device__ __forceinline__ long long sk_begin(int c, long long U, int C) { retur
 // ---------------------------------------------------------------------------
 // tcgen05 / TMA helpers
 
+// PAIR: the ::2 forms, executed by the same warp of both CTAs (the columns are taken in
+// both tensor memories)
+template <bool PAIR>
 __device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot),
-               "r"(ncols)
-               : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  if constexpr (PAIR) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  } else {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
 }
+template <bool PAIR>
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
+  if constexpr (PAIR)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+  else
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -156,20 +202,58 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// Arrive on `bar` once every tcgen05.mma this thread issued before has completed.
+// Arrive on `bar` (a shared::cluster address: this CTA's, or the peer's) once every
+// tcgen05.mma this thread issued before has completed.
+template <bool PAIR>
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
+  if constexpr (PAIR)
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+  else
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
 }
-// D[tmem] (+)= A[smem] . B[smem]^T, both K-major (shape in the instruction descriptor)
+// D[tmem] (+)= A[smem] . B[smem]^T, both K-major (shape in the instruction descriptor).
+// PAIR: issued by the leader CTA; A's rows and B's rows come half from each CTA's shared
+// memory (same offsets), D's rows half into each CTA's tensor memory.
+template <bool PAIR>
 __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u)
-      : "memory");
+  if constexpr (PAIR)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u)
+        : "memory");
+}
+// This CTA's rank in its cluster; the shared::cluster address of this CTA's shared-memory
+// address `a` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t a, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  return r;
+}
+// Arrive on an mbarrier of another CTA of the cluster (release at cluster scope).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
+}
+// Every thread of every CTA of the cluster.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -197,6 +281,16 @@ __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int
                                        uint32_t bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+// The same copy into this CTA's shared memory, its bytes completing on `bar` in either CTA
+// of the pair (a shared::cluster address: the leader's barrier).
+__device__ __forceinline__ void tma_2d_pair(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
       : "memory");
@@ -233,24 +327,55 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // Wait for the phase with parity `parity` of `bar`.  A healthy wait here lasts microseconds;
 // this one gives up after `limit_ns`, or as soon as another role of the CTA has given up
 // (*abort set; the waits of the teardown ignore it), and then sets `bit` in the error word
-// and *abort, and returns false.  Every
-// role leaves its loop on the first failed wait, so a broken pipeline ends the kernel within
-// a few limits instead of one limit per remaining wait.
+// and *abort, and returns false.  Every role leaves its loop on the first failed wait, so a
+// broken pipeline ends the kernel within a few limits instead of one limit per remaining
+// wait.  `cluster`: the phase completes on arrivals from the other CTA of a pair (acquire at
+// cluster scope).
 constexpr uint64_t kWaitNs = 100ull * 1000 * 1000;
-__device__ __noinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
-                                     uint32_t bit, uint64_t limit_ns = kWaitNs,
-                                     bool honor_abort = true, bool patient = false,
-                                     uint32_t backoff_ns = 0) {
+
+// Non-blocking test of the phase (the fast path: the phase has usually completed already).
+__device__ __forceinline__ bool mbar_ready(uint32_t bar, uint32_t parity, bool cluster) {
+  uint32_t done;
+  if (cluster)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+  return done != 0;
+}
+
+__device__ __noinline__ bool tc_wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
+                                          uint32_t bit, uint64_t limit_ns, bool honor_abort,
+                                          bool patient, uint32_t backoff_ns, bool cluster) {
   // The first kSpin rounds poll, sleeping backoff_ns between polls (the pipeline's waits are
   // usually short; the sleep keeps a polling lane from taking the issue slots of the warps
   // that do the work); after that each try_wait may suspend the thread for up to kSuspendNs
   // until the phase completes.  `patient` waiters (the epilogue, whose waits last a whole
-  // tile) suspend from the start.
+  // tile) suspend from the start.  The clock is read only every 64 rounds.
   constexpr uint32_t kSpin = 2048, kSuspendNs = 500;
-  const uint64_t t0 = globaltimer_ns();
+  uint64_t t0 = 0;
   for (uint32_t it = patient ? kSpin : 0;; ++it) {
     uint32_t done;
-    if (it < kSpin) {
+    if (cluster) {
+      asm volatile(
+          "{\n\t.reg .pred p;\n\t"
+          "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}"
+          : "=r"(done)
+          : "r"(bar), "r"(parity)
+          : "memory");
+    } else if (it < kSpin) {
       asm volatile(
           "{\n\t.reg .pred p;\n\t"
           "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -271,12 +396,25 @@ __device__ __noinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile uin
     // past the first polls, sleep between them: leave the issue slots to the working warps
     if (backoff_ns && it >= 256 && it < kSpin) __nanosleep(backoff_ns);
     if ((it & 63u) == 63u) {
-      if ((honor_abort && *abort) || globaltimer_ns() - t0 > limit_ns) break;
+      if (honor_abort && *abort) break;
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0)
+        t0 = now;
+      else if (now - t0 > limit_ns)
+        break;
     }
   }
   atomicOr(&g_tc_err, bit);
   *abort = 1u;
   return false;
+}
+
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
+                                        uint32_t bit, uint64_t limit_ns = kWaitNs,
+                                        bool honor_abort = true, bool patient = false,
+                                        uint32_t backoff_ns = 0, bool cluster = false) {
+  if (mbar_ready(bar, parity, cluster)) return true;
+  return tc_wait_slow(bar, parity, abort, bit, limit_ns, honor_abort, patient, backoff_ns, cluster);
 }
 
 // ---------------------------------------------------------------------------
@@ -290,13 +428,13 @@ struct DqFrag {
   uint32_t p0, p1;  // scale and zero pairs (uniform) | absmax of rows gi, gi + 8 (LUT4)
 };
 
-// The stage's codes and parameters of tile jj, from shared memory (bulk-copied by the TMA
-// lane; layouts as in TcCfg): `st` = the stage, `half` = kb % 2.
+// The stage's codes and parameters of tile jj, from shared memory (tensor-copied by the code
+// producer; layouts as in TcCfg): `cs` = the stage's code slot, `half` = kb % 2.
 template <int FMT, class C>
-__device__ __forceinline__ void dq_load_smem(uint32_t st, int jj, int half, int lane,
+__device__ __forceinline__ void dq_load_smem(uint32_t cs, int jj, int half, int lane,
                                              DqFrag<FMT>& f) {
   const int gi = lane >> 2;
-  const uint32_t c = st + C::kCodeOff + jj * C::kCodeChunk;
+  const uint32_t c = cs + jj * C::kCodeChunk;
   if constexpr (FMT == kW2) {  // the whole chunk: steps 4 half .. 4 half + 3 = words 2 half, +1
     const uint2 v = qlk::lds64(c + lane * 16 + half * 8);
     f.w[0] = v.x;
@@ -317,7 +455,7 @@ __device__ __forceinline__ void dq_load_smem(uint32_t st, int jj, int half, int 
     f.w[2] = v.z;
     f.w[3] = v.w;
   }
-  const uint32_t pa = st + C::kParOff;
+  const uint32_t pa = cs + C::kParOff;
   if constexpr (FMT == kLUT4) {  // absmax of (rows gi, gi + 8) for this half's 64-block
     const uint2 v = qlk::lds64(pa + jj * 128 + gi * 16 + half * 8);
     f.p0 = v.x;
@@ -377,12 +515,12 @@ struct CodeMaps {
   CUtensorMap codes, p0, p1;
 };
 
-template <int BN, bool FUSED, int FMT>
-__global__ void __launch_bounds__(TcCfg<BN, FUSED, FMT>::kThreads, 1)
+template <int BN, bool FUSED, int FMT, bool PAIR>
+__global__ void __launch_bounds__(TcCfg<BN, FUSED, FMT, PAIR>::kThreads, 1)
     prefill_tc_kernel(const TcParams P, const __grid_constant__ CUtensorMap xmap,
                       const __grid_constant__ CUtensorMap wmap,
                       const __grid_constant__ CodeMaps cmaps) {
-  using C = TcCfg<BN, FUSED, FMT>;
+  using C = TcCfg<BN, FUSED, FMT, PAIR>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = qlk::smem_addr(smem_raw);
   const uint32_t ring = (raw + 1023u) & ~1023u;  // the swizzled layout wants 1024-byte atoms
@@ -393,11 +531,31 @@ __global__ void __launch_bounds__(TcCfg<BN, FUSED, FMT>::kThreads, 1)
   auto accf = [&](int a) { return bars + 8 * (2 * C::S + a); };
   auto acce = [&](int a) { return bars + 8 * (2 * C::S + 2 + a); };
   const uint32_t fin = bars + 8 * (2 * C::S + 4);  // the last MMAs' completion
-  auto cfull = [&](int s) { return bars + 8 * (2 * C::S + 5 + s); };  // FUSED: codes landed
+  auto cfull = [&](int c) { return bars + 8 * (2 * C::S + 5 + c); };  // FUSED: codes landed
+  auto cempty = [&](int c) { return bars + 8 * (2 * C::S + 5 + C::SC + c); };  // ... read
   const uint32_t slot = ring + C::kSlotOff;
   volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + C::kSlotOff + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KB = P.K / kBK;
+  // PAIR: rank 0 (the leader) issues the MMAs and owns the barriers of the pair's pipeline
+  // (full, acce); both CTAs copy their own halves of x (and W) and dequantize their own A
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int wk = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;  // worker
+  const int nwk = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  // the leader's barrier `b` as this CTA addresses it; the peer's copy of own barrier `b`
+  auto lead = [&](uint32_t b) { return (PAIR && !leader) ? cluster_addr(b, 0) : b; };
+  auto arrive_lead = [&](uint32_t b) {
+    if (PAIR && !leader)
+      mbar_arrive_remote(cluster_addr(b, 0));
+    else
+      qlk::mbar_arrive(b);
+  };
+  // the leader's commits release both CTAs' barriers
+  auto commit_both = [&](uint32_t b) {
+    tc_commit<PAIR>(b);
+    if constexpr (PAIR) tc_commit<PAIR>(cluster_addr(b, 1));
+  };
 
   __shared__ float lut_s[16];
   if (FUSED && FMT == kLUT4 && threadIdx.x < 16)
@@ -406,29 +564,36 @@ __global__ void __launch_bounds__(TcCfg<BN, FUSED, FMT>::kThreads, 1)
     for (int s = 0; s < C::S; ++s) {
       qlk::mbar_init(full(s), C::kFullCount);
       qlk::mbar_init(empty(s), 1);
-      qlk::mbar_init(cfull(s), 1);
+    }
+    for (int c = 0; c < C::SC; ++c) {
+      qlk::mbar_init(cfull(c), 1);
+      qlk::mbar_init(cempty(c), kDqWarps);
     }
     for (int a = 0; a < 2; ++a) {
       qlk::mbar_init(accf(a), 1);
-      qlk::mbar_init(acce(a), C::kEpiWarps);
+      qlk::mbar_init(acce(a), C::kAccEmptyCount);
     }
     qlk::mbar_init(fin, 1);
     *abort = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) tmem_alloc(slot, C::kTmemCols);
+  if (warp == 1) tmem_alloc<PAIR>(slot, C::kTmemCols);
   tc_fence_before();
-  __syncthreads();
+  // the peer's copies and arrivals reach the leader's barriers only once they are set up
+  if constexpr (PAIR)
+    cluster_sync();
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + C::kSlotOff);
 
   if (warp == 0) {
-    // ---- TMA producer
+    // ---- TMA producer (each CTA its own halves)
     if (lane == 0) {
       int it = 0, t, kb0, kb1;
       bool ok = true;
       SegIter sg;
-      sg.init(P, KB);
+      sg.init(P, KB, wk, nwk);
       while (ok && sg.next(P, KB, t, kb0, kb1)) {
         const int nt = t / P.mtiles, mt = t - nt * P.mtiles;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
@@ -438,72 +603,103 @@ __global__ void __launch_bounds__(TcCfg<BN, FUSED, FMT>::kThreads, 1)
                              false, 64)))
             break;
           const uint32_t st = ring + s * C::kStageBytes;
-          if constexpr (FUSED) {
-            // the stage's packed codes (rows: the block's 8 chunks of the group, columns: the
-            // stage's half, or all of a W2 chunk) and the group's parameters, three tensor
-            // copies; rows past the block are another group's (unused) or read as zeros
-            const int g = kb >> 1, half = kb & 1;
-            const int ch0 = (int)chunk_index(nt, g, 0, P.G, P.ntiles);
-            qlk::mbar_arrive_expect_tx(cfull(s), C::kCodeBytes + C::kParBytes);
-            tma_2d(st + C::kCodeOff, &cmaps.codes, FMT == kW2 ? 0 : half * (C::kCodeChunk / 4), ch0,
-                   cfull(s));
-            if constexpr (FMT == kLUT4) {
-              tma_2d(st + C::kParOff, &cmaps.p1, 0, ch0, cfull(s));
-            } else {
-              tma_2d(st + C::kParOff, &cmaps.p0, 0, ch0, cfull(s));
-              tma_2d(st + C::kParOff + 8 * 32, &cmaps.p1, 0, ch0, cfull(s));
-            }
+          if (leader) qlk::mbar_arrive_expect_tx(full(s), C::kFullBytes);
+          const int xrow = mt * BN + (int)rank * C::kBRows;
+          const int wrow = nt * C::kRows + (int)rank * kBM;
+          if constexpr (PAIR) {
+            tma_2d_pair(st + C::kABytes, &xmap, kb * kBK, xrow, lead(full(s)));
+            if constexpr (!FUSED) tma_2d_pair(st, &wmap, kb * kBK, wrow, lead(full(s)));
+          } else {
+            tma_2d(st + C::kABytes, &xmap, kb * kBK, xrow, full(s));
+            if constexpr (!FUSED) tma_2d(st, &wmap, kb * kBK, wrow, full(s));
           }
-          qlk::mbar_arrive_expect_tx(full(s), C::kBBytes + (FUSED ? 0 : C::kABytes));
-          tma_2d(st + C::kABytes, &xmap, kb * kBK, mt * BN, full(s));
-          if constexpr (!FUSED) tma_2d(st, &wmap, kb * kBK, nt * kBM, full(s));
         }
       }
       // no copy of this CTA is still in flight when it exits: wait for the last stages filled
-      for (int i = (it > C::S ? it - C::S : 0); i < it; ++i) {
-        tc_wait(full(i % C::S), (i / C::S) & 1, abort, kErrStage, kWaitNs / 10, false);
-        if (FUSED) tc_wait(cfull(i % C::S), (i / C::S) & 1, abort, kErrStage, kWaitNs / 10, false);
+      // (the leader's full barriers count the bytes of both CTAs of a pair; the pair meets
+      // at a cluster barrier before either exits)
+      if (leader)
+        for (int i = (it > C::S ? it - C::S : 0); i < it; ++i)
+          tc_wait(full(i % C::S), (i / C::S) & 1, abort, kErrStage, kWaitNs / 10, false);
+    }
+  } else if (FUSED && warp == C::kCodeWarp) {
+    // ---- code producer: the stages' packed codes (rows: the block's 8 chunks of the group,
+    // columns: the stage's half, or all of a W2 chunk) and the group's parameters, three
+    // tensor copies per stage into the code ring; rows past the block are another group's
+    // (unused) or read as zeros
+    if (lane == 0) {
+      int it = 0, t, kb0, kb1;
+      bool ok = true;
+      SegIter sg;
+      sg.init(P, KB, wk, nwk);
+      while (ok && sg.next(P, KB, t, kb0, kb1)) {
+        const int nt = t / P.mtiles;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int c = it % C::SC;
+          if (it >= C::SC &&
+              !(ok = tc_wait(cempty(c), ((it / C::SC) - 1) & 1, abort, kErrStage, kWaitNs, true,
+                             false, 64)))
+            break;
+          const uint32_t cs = ring + C::kCodeRingOff + c * C::kCodeSlot;
+          const int g = kb >> 1, half = kb & 1;
+          const int ch0 = (int)chunk_index(nt * C::kCtas + (int)rank, g, 0, P.G, P.ntiles);
+          qlk::mbar_arrive_expect_tx(cfull(c), C::kCodeBytes + C::kParBytes);
+          tma_2d(cs, &cmaps.codes, FMT == kW2 ? 0 : half * (C::kCodeChunk / 4), ch0, cfull(c));
+          if constexpr (FMT == kLUT4) {
+            tma_2d(cs + C::kParOff, &cmaps.p1, 0, ch0, cfull(c));
+          } else {
+            tma_2d(cs + C::kParOff, &cmaps.p0, 0, ch0, cfull(c));
+            tma_2d(cs + C::kParOff + 8 * 32, &cmaps.p1, 0, ch0, cfull(c));
+          }
+        }
       }
+      // no copy in flight when the CTA exits
+      for (int i = (it > C::SC ? it - C::SC : 0); i < it; ++i)
+        tc_wait(cfull(i % C::SC), (i / C::SC) & 1, abort, kErrStage, kWaitNs / 10, false);
     }
   } else if (warp == 1) {
-    // ---- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16(kBM, BN);
+    // ---- MMA issuer (the leader of a pair)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_f16(C::kRows, BN);
       int it = 0, j = 0, t, kb0, kb1;
       bool ok = true;
       SegIter sg;
-      sg.init(P, KB);
+      sg.init(P, KB, wk, nwk);
       for (; ok && sg.next(P, KB, t, kb0, kb1); ++j) {
         const int a = j & 1;
-        if (j >= 2 && !(ok = tc_wait(acce(a), ((j >> 1) - 1) & 1, abort, kErrAcc))) break;
+        if (j >= 2 &&
+            !(ok = tc_wait(acce(a), ((j >> 1) - 1) & 1, abort, kErrAcc, kWaitNs, true, false, 0, PAIR)))
+          break;
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(a * BN);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % C::S;
-          if (!(ok = tc_wait(full(s), (it / C::S) & 1, abort, kErrStage, kWaitNs, true, false, 32)))
+          if (!(ok = tc_wait(full(s), (it / C::S) & 1, abort, kErrStage, kWaitNs, true, false, 32,
+                             PAIR && FUSED)))
             break;
           tc_fence_after();
           const uint32_t st = ring + s * C::kStageBytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            tc_mma(d, desc_sw128(st + 32 * kk), desc_sw128(st + C::kABytes + 32 * kk), idesc,
-                   (kb != kb0) || (kk != 0));
-          tc_commit(empty(s));  // the stage is free once these MMAs have read it
+            tc_mma<PAIR>(d, desc_sw128(st + 32 * kk), desc_sw128(st + C::kABytes + 32 * kk), idesc,
+                         (kb != kb0) || (kk != 0));
+          commit_both(empty(s));  // the stage is free once these MMAs have read it
         }
-        if (ok) tc_commit(accf(a));  // the segment's accumulator is complete
+        if (ok) commit_both(accf(a));  // the segment's accumulator is complete
       }
-      // every MMA issued has completed before the tensor memory is released
-      tc_commit(fin);
+      // every MMA issued has completed before the tensor memory is released (the peer
+      // releases its columns after the cluster barrier below, which the leader reaches
+      // only after this wait)
+      tc_commit<PAIR>(fin);
       tc_wait(fin, 0, abort, kErrAcc, kWaitNs / 10, false);
     }
   } else if (warp < C::kDqWarp0) {
-    // ---- epilogue: warp w reads accumulator lanes 32 (w % 4) .. + 31 (weight rows)
+    // ---- epilogue: warp w reads accumulator lanes 32 (w % 4) .. + 31 (this CTA's weight rows)
     const int q = warp & 3;
     const long long U = (long long)P.tiles * KB;
-    const int Cg = gridDim.x;
     int j = 0, t, kb0, kb1;
     SegIter sg;
-    sg.init(P, KB);
+    sg.init(P, KB, wk, nwk);
     for (; sg.next(P, KB, t, kb0, kb1); ++j) {
       const int a = j & 1;
       const int nt = t / P.mtiles, mt = t - nt * P.mtiles;
@@ -512,7 +708,7 @@ __global__ void __launch_bounds__(TcCfg<BN, FUSED, FMT>::kThreads, 1)
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       tc_fence_after();
       const int row = 32 * q + lane;
-      const int n = nt * kBM + row;
+      const int n = nt * C::kRows + (int)rank * kBM + row;
       const int m0 = mt * BN;
       const int cols = (P.M - m0) < BN ? (P.M - m0) : BN;
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * BN);
@@ -529,13 +725,13 @@ __global__ void __launch_bounds__(TcCfg<BN, FUSED, FMT>::kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) qlk::mbar_arrive(acce(a));
+        if (lane == 0) arrive_lead(acce(a));
         continue;
       }
       // part of a tile (stream-K): publish this CTA's fp32 partial; the last contributor
-      // adds all of them in CTA order and stores y (nobody waits for anybody)
-      const int slot = 2 * (int)blockIdx.x + (j == 0 ? 0 : 1);
-      float* mine = P.partials + ((size_t)slot * kBM + row) * BN;
+      // adds all of them in worker order and stores y (nobody waits for anybody)
+      const int pslot = 2 * (int)blockIdx.x + (j == 0 ? 0 : 1);
+      float* mine = P.partials + ((size_t)pslot * kBM + row) * BN;
       for (int c0 = 0; c0 < cols; c0 += 16) {
         uint32_t r[16];
         tmem_ld16(tbase + (uint32_t)c0, r);
@@ -546,11 +742,12 @@ __global__ void __launch_bounds__(TcCfg<BN, FUSED, FMT>::kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) qlk::mbar_arrive(acce(a));  // the accumulator is free again
-      const int cf = sk_cta_of((long long)t * KB, U, Cg);
-      const int cl = sk_cta_of((long long)(t + 1) * KB - 1, U, Cg);
+      if (lane == 0) arrive_lead(acce(a));  // the accumulator is free again
+      const int cf = sk_cta_of((long long)t * KB, U, nwk);
+      const int cl = sk_cta_of((long long)(t + 1) * KB - 1, U, nwk);
+      uint32_t* counter = P.counters + ((size_t)t * C::kCtas + rank) * 4 + q;
       uint32_t prev = 0;
-      if (lane == 0) prev = qlk::arrive_acq_rel(P.counters + (size_t)t * 4 + q);
+      if (lane == 0) prev = qlk::arrive_acq_rel(counter);
       prev = __shfl_sync(0xffffffffu, prev, 0);
       if (prev + 1 != (uint32_t)(cl - cf + 1)) continue;
       __syncwarp();
@@ -559,7 +756,8 @@ __global__ void __launch_bounds__(TcCfg<BN, FUSED, FMT>::kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e) acc[e] = 0.f;
         for (int cc = cf; cc <= cl; ++cc) {
-          const int sl = (sk_begin(cc, U, Cg) >= (long long)t * KB) ? 2 * cc : 2 * cc + 1;
+          const int cta = cc * C::kCtas + (int)rank;
+          const int sl = (sk_begin(cc, U, nwk) >= (long long)t * KB) ? 2 * cta : 2 * cta + 1;
           const float* src = P.partials + ((size_t)sl * kBM + row) * BN + c0;
 #pragma unroll
           for (int e = 0; e < 16; e += 4) {
@@ -576,41 +774,56 @@ __global__ void __launch_bounds__(TcCfg<BN, FUSED, FMT>::kThreads, 1)
             if (c0 + e < cols) P.y[(size_t)(m0 + c0 + e) * P.N + n] = __float2half_rn(acc[e]);
         }
       }
-      if (lane == 0) P.counters[(size_t)t * 4 + q] = 0u;  // ready for the next call
+      if (lane == 0) *counter = 0u;  // ready for the next call
     }
   } else if constexpr (FUSED) {
-    // ---- dequantizing producers: warp dw fills rows 16 dw .. 16 dw + 15 of A from the
-    // codes the TMA lane brought into the same stage
+    // ---- dequantizing producers: warp dw fills rows 16 dw .. 16 dw + 15 of this CTA's A of
+    // stage s (once the MMAs are done with it) from the codes in code slot c, then releases
+    // both
     const int dw = warp - C::kDqWarp0;
     int it = 0, t, kb0, kb1;
     bool ok = true;
     SegIter sg;
-    sg.init(P, KB);
+    sg.init(P, KB, wk, nwk);
     while (ok && sg.next(P, KB, t, kb0, kb1)) {
-      const int tb = tiles_in_block(t / P.mtiles, P.ntiles);
+      // tiles of this CTA's 128-row block (none for a block past N)
+      const int blk = (t / P.mtiles) * C::kCtas + (int)rank;
+      const int tb = blk * kBlockTiles < P.ntiles ? tiles_in_block(blk, P.ntiles) : 0;
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
-        const int s = it % C::S;
-        if (lane == 0)
-          ok = tc_wait(cfull(s), (it / C::S) & 1, abort, kErrStage, kWaitNs, true, false, 32);
+        const int s = it % C::S, c = it % C::SC;
+        if (lane == 0) {
+          ok = tc_wait(cfull(c), (it / C::SC) & 1, abort, kErrStage, kWaitNs, true, false, 32);
+          if (ok && it >= C::S)
+            ok = tc_wait(empty(s), ((it / C::S) - 1) & 1, abort, kErrStage, kWaitNs, true, false, 32);
+        }
         if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
         const uint32_t st = ring + s * C::kStageBytes;
-        if (dw < tb) {
-          DqFrag<FMT> f;
-          dq_load_smem<FMT, C>(st, dw, kb & 1, lane, f);
-          dq_store<FMT>(f, st, dw, lane, lut_s);
-        }
+        DqFrag<FMT> f;
+        if (dw < tb) dq_load_smem<FMT, C>(ring + C::kCodeRingOff + c * C::kCodeSlot, dw, kb & 1, lane, f);
+        if (dw < tb) dq_store<FMT>(f, st, dw, lane, lut_s);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the MMAs
         __syncwarp();
-        if (lane == 0) qlk::mbar_arrive(full(s));
+        // the code slot is released only now, once every lane has used the words it read
+        // (releasing it right after the shared loads and a __syncwarp let the next copy
+        // overwrite words some lanes had not yet read: wrong results in a stress run)
+        if (lane == 0) {
+          qlk::mbar_arrive(cempty(c));
+          arrive_lead(full(s));
+        }
       }
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  // PAIR: neither CTA exits (or releases its tensor memory) while the other may still
+  // arrive on its barriers or the leader's MMAs may still use its memory
+  if constexpr (PAIR)
+    cluster_sync();
+  else
+    __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
+    tmem_dealloc<PAIR>(tmem, C::kTmemCols);
   }
 }
 
@@ -660,33 +873,58 @@ bool encode_rows(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool FUSED, int FMT>
+// Workers (CTAs, or cluster pairs) that are resident at once on this device, per instance.
+template <int BN, bool FUSED, int FMT, bool PAIR>
+int resident_workers(int dev, int sms) {
+  using C = TcCfg<BN, FUSED, FMT, PAIR>;
+  auto fn = prefill_tc_kernel<BN, FUSED, FMT, PAIR>;
+  static std::mutex mu;
+  static std::unordered_map<int, int> known;
+  std::lock_guard<std::mutex> lk(mu);
+  auto k = known.find(dev);
+  if (k != known.end()) return k->second;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+      cudaSuccess)
+    return 0;
+  int n = 0;
+  if constexpr (PAIR) {
+    // pairs must sit on two SMs of one GPC: count the clusters that fit, not SMs / 2
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) n = 0;
+  } else {
+    int occ = 0;  // the CTA (threads x registers, shared memory) must fit on an SM
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, C::kThreads, C::kSmemBytes) ==
+            cudaSuccess &&
+        occ >= 1)
+      n = sms;
+  }
+  if (n > 0) known[dev] = n;
+  return n;
+}
+
+template <int BN, bool FUSED, int FMT, bool PAIR>
 ql_status launch_tc(const TcParams& P, const void* x, const void* w, cudaStream_t st) {
-  using C = TcCfg<BN, FUSED, FMT>;
-  auto fn = prefill_tc_kernel<BN, FUSED, FMT>;
+  using C = TcCfg<BN, FUSED, FMT, PAIR>;
+  auto fn = prefill_tc_kernel<BN, FUSED, FMT, PAIR>;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QL_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return QL_ERR_CUDA;
-  {
-    static std::mutex mu;
-    static std::unordered_map<int, bool> ready;
-    std::lock_guard<std::mutex> lk(mu);
-    if (!ready[dev]) {
-      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
-          cudaSuccess)
-        return QL_ERR_CUDA;
-      int occ = 0;  // the CTA (threads x registers, shared memory) must fit on an SM
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, C::kThreads, C::kSmemBytes) !=
-              cudaSuccess ||
-          occ < 1)
-        return QL_ERR_CUDA;
-      ready[dev] = true;
-    }
-  }
+  const int maxw = resident_workers<BN, FUSED, FMT, PAIR>(dev, sms);
+  if (maxw <= 0) return QL_ERR_CUDA;
   CUtensorMap xmap, wmap;
   CodeMaps cm;
-  if (!encode_kmajor(&xmap, x, P.M, P.K, BN)) return QL_ERR_CUDA;
+  if (!encode_kmajor(&xmap, x, P.M, P.K, C::kBRows)) return QL_ERR_CUDA;
   if (FUSED) {
     wmap = xmap;  // unused
     const long long nchunks = (long long)P.ntiles * P.G;
@@ -707,18 +945,48 @@ ql_status launch_tc(const TcParams& P, const void* x, const void* w, cudaStream_
   } else {
     cm.codes = cm.p0 = cm.p1 = xmap;  // unused
   }
-  // stream-K: one CTA per SM (at most one per k-block, so that every CTA has work: the
-  // fix-up counts the CTAs whose ranges meet a tile), the k-blocks shared out evenly; whole
-  // tiles: at most one CTA per tile
+  // stream-K: one worker per SM (pair of SMs), at most one per k-block, so that every worker
+  // has work (the fix-up counts the workers whose ranges meet a tile), the k-blocks shared out
+  // evenly; whole tiles: at most one worker per tile
   const long long units = P.partials ? (long long)P.tiles * (P.K / kBK) : P.tiles;
-  const int grid = units < sms ? (int)units : sms;
-  fn<<<grid, C::kThreads, C::kSmemBytes, st>>>(P, xmap, wmap, cm);
+  const int workers = units < maxw ? (int)units : maxw;
+  if constexpr (PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * workers, 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = st;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, fn, P, xmap, wmap, cm) != cudaSuccess) return QL_ERR_CUDA;
+  } else {
+    fn<<<workers, C::kThreads, C::kSmemBytes, st>>>(P, xmap, wmap, cm);
+  }
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+}
+
+// Tile form: the dense GEMM on cluster pairs (tcgen05 cta_group::2: each CTA copies half of
+// the tile's x, which the dense GEMM's L2 traffic and power budget favour), the fused one on
+// single CTAs (its dequantizing warps would otherwise also wait for the other CTA's).  Both
+// measured on 8192 x 28672 at M = 512 and 2048.  QLINEAR_TC_PAIR = 0 / 1 forces one form.
+bool use_pair(bool fused) {
+  const char* e = getenv("QLINEAR_TC_PAIR");
+  if (e && (e[0] == '0' || e[0] == '1')) return e[0] == '1';
+  return !fused;
 }
 
 template <bool FUSED, int FMT>
 ql_status launch_bn(const TcParams& P, const void* x, const void* w, cudaStream_t st) {
-  return P.M <= 128 ? launch_tc<128, FUSED, FMT>(P, x, w, st) : launch_tc<256, FUSED, FMT>(P, x, w, st);
+  if (P.pair)
+    return P.M <= 128 ? launch_tc<128, FUSED, FMT, true>(P, x, w, st)
+                      : launch_tc<256, FUSED, FMT, true>(P, x, w, st);
+  return P.M <= 128 ? launch_tc<128, FUSED, FMT, false>(P, x, w, st)
+                    : launch_tc<256, FUSED, FMT, false>(P, x, w, st);
 }
 
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
@@ -735,22 +1003,25 @@ TcParams make_params(const void* packed, const void* p0, const void* p1, void* y
   P.K = K;
   P.G = K / kGroup;
   P.ntiles = N / kTileN;
+  P.pair = use_pair(packed != nullptr);
   const int bn = M <= 128 ? 128 : 256;
+  const int rows = P.pair ? 2 * kBM : kBM;
   P.mtiles = (M + bn - 1) / bn;
-  P.tiles = ((N + kBM - 1) / kBM) * P.mtiles;
+  P.tiles = ((N + rows - 1) / rows) * P.mtiles;
   P.partials = nullptr;
   P.counters = nullptr;
   return P;
 }
 
-// Workspace of the stream-K schedule: arrival counters (one per tile and epilogue warp, zero
-// between calls) and two fp32 partial tiles (128 x BN) per CTA.
+// Workspace of the stream-K schedule: arrival counters (one per tile, CTA of the tile and
+// epilogue warp; zero between calls; sized for 256-row tiles of two CTAs, which is at least
+// the count for 128-row tiles) and two fp32 partial tiles (128 x BN) per CTA.
 struct SkLayout {
   size_t counter_bytes, partial_offset, bytes;
 };
 SkLayout sk_layout(int M, int N, int sms) {
   const int bn = M <= 128 ? 128 : 256;
-  const long long tiles = (long long)((N + kBM - 1) / kBM) * ((M + bn - 1) / bn);
+  const long long tiles = (long long)((N + 2 * kBM - 1) / (2 * kBM)) * 2 * ((M + bn - 1) / bn);
   SkLayout L;
   L.counter_bytes = (size_t)tiles * 4 * sizeof(uint32_t);
   L.partial_offset = (L.counter_bytes + 255) / 256 * 256;
