@@ -80,7 +80,15 @@ typedef enum {
   QL_ERR_LIBRARY = 7      /* reserved (no library is opened at run time) */
 } ql_status;
 
-typedef enum { QL_FMT_W2 = 2, QL_FMT_W3 = 3, QL_FMT_W4 = 4, QL_FMT_W8 = 8, QL_FMT_LUT4 = 16 } ql_format;
+typedef enum {
+  QL_FMT_W2 = 2,
+  QL_FMT_W3 = 3,
+  QL_FMT_W4 = 4,
+  QL_FMT_W8 = 8,
+  QL_FMT_LUT4 = 16,
+  QL_FMT_CB = 32 /* m1v4g128 codebook, tensor-core layout (qlinear_codebook_tc): for
+                    qlinear_workspace_bytes and qlinear_plan only */
+} ql_format;
 
 /* Opaque stream handle, ABI-compatible with cudaStream_t. */
 typedef struct CUstream_st* ql_stream_t;
@@ -347,6 +355,30 @@ size_t qlinear_codebook_workspace_bytes(int M, int N, int K);
 ql_status qlinear_codebook(const uint16_t* x, const uint8_t* codes, const uint16_t* scales,
                            const uint16_t* codebook, uint16_t* y, int M, int N, int K,
                            void* workspace, size_t workspace_bytes, ql_stream_t stream);
+
+/* The same product on the tensor cores, through the GEMV kernel (qlinear_w2a16's pipeline,
+ * stream-K grid and split-K fix-up): the codebook's 256 vectors are copied 16 times into
+ * shared memory, and each tensor-core step takes, per lane, one 8-byte vector for each of
+ * its two weight rows as the A fragment (the step's four k per lane are one vector).  The
+ * Psumbook form (qlinear_codebook) follows the CodeGEMM page; this form reaches the same
+ * sums with one lookup per 4 weights and row instead of one per 4 weights, row and token,
+ * which on B200 is the faster use of shared memory (measured).
+ *   codes    : packed by qlinear_pack_codebook_tc, 32-byte aligned;
+ *   scales   : fp16 [K / 128][N] packed by qlinear_pack_params(QL_FMT_W4, ...), 16-byte
+ *              aligned (the uniform formats' scale layout);
+ *   codebook : fp16 [256][4], 8-byte aligned;
+ *   x, y     : as qlinear_w4a16 (M <= 16, N % 16 == 0, K % 128 == 0);
+ *   workspace: qlinear_workspace_bytes(QL_FMT_CB, M, N, K) bytes, as for qlinear_w4a16.
+ * fp32 accumulation, y rounded once to fp16; reproducible. */
+ql_status qlinear_codebook_tc(const uint16_t* x, const uint8_t* codes, const uint16_t* scales,
+                              const uint16_t* codebook, uint16_t* y, int M, int N, int K,
+                              void* workspace, size_t workspace_bytes, ql_stream_t stream);
+
+/* Canonical codes uint8 [K / 4][N] into the layout of qlinear_codebook_tc: the chunk order
+ * of the uniform formats (16-column tiles by 128-k groups), 512 bytes per chunk, lane l's
+ * 16 bytes at 16 l, byte 2 s + r of them the code of step s for row (tile column) l / 4 + 8 r.
+ * Host buffers of K / 4 * N bytes. */
+ql_status qlinear_pack_codebook_tc(const uint8_t* codes, uint8_t* packed, int N, int K);
 
 /* ---------------------------------------------------------------------------
  * Measured policy map and dispatcher.

@@ -296,3 +296,36 @@ def test_workspace_too_small_is_rejected():
     with pytest.raises(ql.QLinearError) as e:
         lay.forward(torch.zeros((1, K), dtype=torch.float16, device=DEV))
     assert e.value.status == 5
+
+
+@pytest.mark.parametrize("kind,M", [("w4", 1), ("w2", 1), ("w4", 16), ("lut4", 1), ("outlier", 8)])
+def test_many_launches_bit_identical(kind, M):
+    """A stage refilled before every lane has read it would show as results that differ
+    between launches: 200 back-to-back launches on a layer whose CTAs each stream many units
+    (every ring wraps), all bit-identical to the first, the first within tolerance."""
+    K, N = 4096, 2048
+    x, xd = _x(773 + M, M, K)
+    if kind == "lut4":
+        L = lut4_layer(770, K, N)
+        lay = layers.from_lut4(L, DEV)
+        want = oracle.gemv_lut4(x, L.qbytes, L.lut, L.absmax, 64)
+    elif kind == "outlier":
+        o = outlier_layer(771, K, N)
+        lay = layers.from_outlier(o, DEV)
+        want = oracle.gemv_outlier(x, o.dense.qweight, o.dense.scales, o.dense.zeros,
+                                   o.tile_offsets, o.tile_rc, o.tile_vals, 4, 128)
+    else:
+        bits = int(kind[1:])
+        u = uniform_layer(772, K, N, bits)
+        lay = layers.from_uniform(u, DEV)
+        want = oracle.gemv_uniform(x, u.qweight, u.scales, u.zeros, bits, 128)
+    y = torch.empty((M, N), dtype=torch.float16, device=DEV)
+    lay.forward(xd, y)
+    torch.cuda.synchronize()
+    first = y.view(torch.int16).cpu().numpy().copy()
+    assert_parity(first.view(np.float16).astype(np.float64), want, what=f"{kind} M={M}")
+    for _ in range(200):
+        lay.forward(xd, y)
+        torch.cuda.synchronize()
+        assert np.array_equal(y.view(torch.int16).cpu().numpy(), first)
+    assert lay.read_error() == 0

@@ -274,3 +274,29 @@ def test_w3_packer_planes(ql):
     assert lib.qlinear_w3a16(None, a, a, a, a, 1, 128, 128, 128, a, 1 << 20, None) == 1
     assert ql.qlinear_params_bytes_grouped(3, 64, N, K) == 0
     assert ql.qlinear_params_bytes_grouped(3, K, N, K) == G * N * 2
+
+
+def test_pack_codebook_tc_layout(ql):
+    """Byte 2 s + r of lane l in chunk (block b, group g, tile jj) is the code of the 4-vector
+    that holds k = 128 g + 32 (s // 2) + 8 (l % 4) + 4 (s % 2) of column
+    16 (8 b + jj) + l // 4 + 8 r (the fragment k order of the GEMV)."""
+    K, N = 256, 160  # 2 groups, 10 tiles: a full block and a ragged one of 2 tiles
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 256, size=(K // 4, N), dtype=np.uint8)
+    packed = ql.qlinear_pack_codebook_tc(codes, N, K)
+    G, ntiles = K // 128, N // 16
+    seen = 0
+    for b in range(2):
+        tb = min(8, ntiles - 8 * b)
+        for g in range(G):
+            for jj in range(tb):
+                c = b * G * 8 + g * tb + jj
+                for lane in (0, 5, 18, 31):
+                    for s in range(8):
+                        for r in range(2):
+                            k = 128 * g + 32 * (s // 2) + 8 * (lane % 4) + 4 * (s % 2)
+                            n = 16 * (8 * b + jj) + lane // 4 + 8 * r
+                            assert packed[c * 512 + lane * 16 + 2 * s + r] == codes[k // 4, n]
+                            seen += 1
+    assert seen == (8 + 2) * G * 4 * 16
+    assert sorted(packed.tolist()) == sorted(codes.ravel().tolist())  # a permutation

@@ -27,6 +27,7 @@ if not os.path.exists(LIBRARY_PATH):
 _lib = ctypes.CDLL(LIBRARY_PATH)
 
 QL_FMT_W2, QL_FMT_W3, QL_FMT_W4, QL_FMT_W8, QL_FMT_LUT4 = 2, 3, 4, 8, 16
+QL_FMT_CB = 32  # the codebook in the tensor-core layout (workspace and plan queries)
 FORMATS = {"w2": QL_FMT_W2, "w3": QL_FMT_W3, "w4": QL_FMT_W4, "w8": QL_FMT_W8,
            "lut4": QL_FMT_LUT4}
 STATUS = {0: "QL_OK", 1: "QL_ERR_NULL", 2: "QL_ERR_SHAPE", 3: "QL_ERR_ALIGN",
@@ -90,6 +91,8 @@ _SIGS = {
     "qlinear_pack_codebook_scales": (_I, [_P, _P, _I, _I]),
     "qlinear_codebook_workspace_bytes": (_SZ, [_I, _I, _I]),
     "qlinear_codebook": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _SZ, _P]),
+    "qlinear_pack_codebook_tc": (_I, [_P, _P, _I, _I]),
+    "qlinear_codebook_tc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _SZ, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -419,4 +422,25 @@ def qlinear_codebook(x, codes, scales, codebook, y, M, N, K, workspace, stream=N
                                K, _ptr(workspace), workspace.numel() * workspace.element_size()
                                if workspace is not None else 0, _stream(stream))
     _check(st, "qlinear_codebook")
+    return y
+
+
+# codebook GEMV on the tensor cores (the GEMV kernel, codebook lookups as A fragments)
+
+
+def qlinear_pack_codebook_tc(codes: np.ndarray, N: int, K: int) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    if codes.size != K // 4 * N:
+        raise QLinearError(2, "qlinear_pack_codebook_tc")
+    out = np.empty(codes.size, dtype=np.uint8)
+    _check(_lib.qlinear_pack_codebook_tc(_np_ptr(codes), _np_ptr(out), N, K),
+           "qlinear_pack_codebook_tc")
+    return out
+
+
+def qlinear_codebook_tc(x, codes, scales, codebook, y, M, N, K, workspace, stream=None):
+    st = _lib.qlinear_codebook_tc(_ptr(x), _ptr(codes), _ptr(scales), _ptr(codebook), _ptr(y), M,
+                                  N, K, _ptr(workspace), workspace.numel() * workspace.element_size()
+                                  if workspace is not None else 0, _stream(stream))
+    _check(st, "qlinear_codebook_tc")
     return y

@@ -104,6 +104,12 @@ template <> struct Fmt<kW8> {
   static constexpr float kHiScale = 1.0f;
   static constexpr int kStagesPerWarpM8 = 1;
 };
+template <> struct Fmt<kCB> {  // 8-bit codebook indices, two per step (rows gi, gi + 8)
+  static constexpr int kWords = 4;
+  static constexpr uint32_t kOnesHi = 0;
+  static constexpr float kHiScale = 1.0f;
+  static constexpr int kStagesPerWarpM8 = 2;
+};
 template <> struct Fmt<kLUT4> {
   static constexpr int kWords = 8;
   static constexpr uint32_t kOnesHi = 0;
@@ -152,11 +158,12 @@ struct Cfg {
   // CTAs per SM the registers are sized for: OCC_, else the format's default (more CTAs,
   // fewer registers per thread)
   static constexpr int kOcc = OCC_;
-  static constexpr int kMinCtas = OCC_ ? OCC_ : (FMT == kLUT4) ? 2 : (MT == 1 && FMT != kW8) ? 3 : 2;
+  static constexpr int kMinCtas =
+      OCC_ ? OCC_ : (FMT == kLUT4 || FMT == kCB) ? 2 : (MT == 1 && FMT != kW8) ? 3 : 2;
   static constexpr int kChunkBytes = 128 * KW;
   static constexpr int kCodeBytes = kBlockTiles * kChunkBytes;
   static constexpr int kParamChunk = (FMT == kLUT4) ? 128 : 32 * NS;   // per tile, per array
-  static constexpr int kParamBytes = (FMT == kLUT4) ? 8 * 128 : 2 * 8 * 32 * NS;
+  static constexpr int kParamBytes = (FMT == kLUT4) ? 8 * 128 : (FMT == kCB) ? 8 * 32 : 2 * 8 * 32 * NS;
   static constexpr int kZeroOff = 8 * 32 * NS;   // zeros after the 8 tiles' scales
   // x rows in a stage: the 2-D tile copy (M >= 2) writes them densely; the single-row
   // kernel keeps 16 bytes of padding, which spreads the fragment loads over the banks
@@ -167,7 +174,8 @@ struct Cfg {
   static constexpr int kRingBytes = S * kStageBytes;
   static constexpr int kBarOff = kRingBytes;                       // full[S], empty[S]
   static constexpr int kLutOff = align_to(kBarOff + 16 * S, 128);
-  static constexpr int kLutBytes = (FMT == kLUT4) ? 256 * 32 * 4 : 0;
+  // LUT4: 256 fp16 pairs x 32 copies; CB: the 256 fp16 4-vectors x 16 copies
+  static constexpr int kLutBytes = (FMT == kLUT4) ? 256 * 32 * 4 : (FMT == kCB) ? 256 * 16 * 8 : 0;
   static constexpr int kRedOff = kLutOff + kLutBytes;              // per-warp block sums
   // each warp holds kTW tiles.  The W4 M <= 8 variants (1, 2 or 4 warps per unit) all size
   // it for kTW = 8, so that they ask for the same shared memory: consecutive launches of
@@ -387,6 +395,15 @@ __device__ __forceinline__ void frag_lut(uint32_t v, uint32_t tbl_lane, uint32_t
   }
 }
 
+// CB: entry (code, copy) at (16 code + copy) * 8 bytes, 16 copies of each 8-byte 4-vector;
+// lane l reads copy l % 16, so the two 16-lane halves of a 64-bit load each touch all 32
+// banks once.
+__device__ __forceinline__ void build_cb_table(uint2* tbl, const __half* codebook, int tid,
+                                               int nthreads) {
+  const uint2* cb = reinterpret_cast<const uint2*>(codebook);
+  for (int e = tid; e < 256 * 16; e += nthreads) tbl[e] = cb[e >> 4];
+}
+
 __device__ __forceinline__ void build_lut_table(uint32_t* tbl, const __half* lut16, int tid,
                                                 int nthreads) {
   for (int e = tid; e < 256 * 32; e += nthreads) {
@@ -419,6 +436,7 @@ struct Gemv {
   static constexpr int NC = C_::NC, T = C_::T, KW = C_::KW, NACC = C_::NACC, S = C_::S;
   static constexpr int WPU = C_::WPU, NP = C_::NP, kTW = C_::kTW;
   static constexpr bool kLut = (FMT == kLUT4);
+  static constexpr bool kCb = (FMT == kCB);
   static constexpr int kBT = kBlockTiles;
 
   // x fragments of one unit (rows gi and, for MT == 2, gi + 8), from the stage.
@@ -465,7 +483,7 @@ struct Gemv {
                               __uint_as_float(a.w));
       } else {
         r.p0[i] = lds32(st + C_::kCodeBytes + (j0 + i) * 32 + gi * 4);
-        r.p1[i] = lds32(st + C_::kCodeBytes + 256 + (j0 + i) * 32 + gi * 4);
+        if constexpr (!kCb) r.p1[i] = lds32(st + C_::kCodeBytes + 256 + (j0 + i) * 32 + gi * 4);
       }
     }
   }
@@ -504,6 +522,49 @@ struct Gemv {
 #pragma unroll
           for (int e = 0; e < NACC; ++e)
             if (!C_::M1 || !(e & 1)) acc[i][e] = fmaf((e & 2) ? a8 : a0, c[i][e], acc[i][e]);
+        }
+      }
+    } else if constexpr (kCb) {
+      // Codebook: in step s the lane's fragment covers the 4 consecutive k of one codebook
+      // vector for row gi (a0, a2) and one for row gi + 8 (a1, a3) (the fragments' k order
+      // is the one x is staged in: real k = 32 (s / 2) + 8 t + 4 (s % 2) + 0..3).  Byte
+      // 2 s + r8 of the lane's 16 code bytes indexes the vector; one 64-bit lookup in the
+      // lane's copy of the table gives both registers of a row.
+      const uint32_t tl = lut + 8u * (uint32_t)(lane & 15);
+      float c[kQ][NACC];
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const int p = s >> 1, h = s & 1;
+        const uint32_t b0 = h ? xr[p].z : xr[p].x, b1 = h ? xr[p].w : xr[p].y;
+        uint32_t b2 = 0, b3 = 0;
+        if constexpr (MT == 2) {
+          b2 = h ? xr2[p].z : xr2[p].x;
+          b3 = h ? xr2[p].w : xr2[p].y;
+        }
+#pragma unroll
+        for (int i = 0; i < kQ; ++i) {
+          const uint32_t v = w[i][s >> 1];
+          uint32_t c0, c1;
+          asm("prmt.b32 %0, %1, 0, %2;" : "=r"(c0) : "r"(v), "r"(0x4440u | (uint32_t)(2 * h)));
+          asm("prmt.b32 %0, %1, 0, %2;" : "=r"(c1) : "r"(v), "r"(0x4440u | (uint32_t)(2 * h + 1)));
+          const uint2 r0 = lds64(c0 * 128u + tl), r1 = lds64(c1 * 128u + tl);
+          const uint32_t a[4] = {r0.x, r1.x, r0.y, r1.y};
+          if (s == 0) {
+            hmma0(&c[i][0], a, b0, b1);
+            if constexpr (MT == 2) hmma0(&c[i][4], a, b2, b3);
+          } else {
+            hmma(&c[i][0], a, b0, b1);
+            if constexpr (MT == 2) hmma(&c[i][4], a, b2, b3);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kQ; ++i) {
+        const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&r.p0[i]));
+#pragma unroll
+        for (int e = 0; e < NACC; ++e) {
+          if (C_::M1 && (e & 1)) continue;  // batch column 1 of the fragment: no such row
+          acc[i][e] = fmaf((e & 2) ? s2.y : s2.x, c[i][e], acc[i][e]);
         }
       }
     } else if constexpr (FMT == kW3) {
@@ -669,7 +730,7 @@ struct Gemv {
         }
 #pragma unroll
       for (int e = 0; e < NACC; ++e)
-        if (!kLut) v[i][e] *= (e & 2) ? kTwo24 * Fmt<FMT>::kHiScale : kTwo24;
+        if (!kLut && !kCb) v[i][e] *= (e & 2) ? kTwo24 * Fmt<FMT>::kHiScale : kTwo24;
     }
     if constexpr (OUTL) {  // the outlier sums of this warp's tiles, then cleared
       const int gi = lane >> 2, t4 = lane & 3;
@@ -779,9 +840,11 @@ struct Gemv {
       const uint32_t full = bars + 8 * s;
       const uint32_t code_bytes = tb * C_::kChunkBytes;
       const uint32_t param_bytes = tb * C_::kParamChunk;
-      mbar_arrive_expect_tx(full, code_bytes + (kLut ? 1 : 2) * param_bytes + 256u * P.M);
+      mbar_arrive_expect_tx(full, code_bytes + (kLut || kCb ? 1 : 2) * param_bytes + 256u * P.M);
       bulk_g2s(st, P.qw + ch * C_::kChunkBytes, code_bytes, full, pol);
-      if constexpr (kLut) {
+      if constexpr (kCb) {  // the scales only
+        bulk_g2s(st + C_::kCodeBytes, P.sc + ch * 16, param_bytes, full, pol);
+      } else if constexpr (kLut) {
         bulk_g2s(st + C_::kCodeBytes, static_cast<const float*>(P.zp) + ch * 32, param_bytes, full,
                  pol);
       } else {
@@ -890,7 +953,7 @@ struct Gemv {
     const uint32_t empty = bars + 8 * (S + s);
     float cx[NACC];
     auto sum_x = [&]() {
-      if constexpr (kLut) {
+      if constexpr (kLut || kCb) {  // no zero points: no sum of x
 #pragma unroll
         for (int e = 0; e < NACC; ++e) cx[e] = 0.f;
       } else {  // sum of x over the group, in the row scales of the codes
@@ -1167,6 +1230,10 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, OUTL, WPU, M1, OCC, NS>::kThreads
   if constexpr (G_::kLut) {
     build_lut_table(reinterpret_cast<uint32_t*>(smem + C_::kLutOff), P.sc, threadIdx.x,
                     C_::kThreads);
+  }
+  if constexpr (G_::kCb) {  // the codebook (fp16 [256][4]) arrives in P.zp
+    build_cb_table(reinterpret_cast<uint2*>(smem + C_::kLutOff), static_cast<const __half*>(P.zp),
+                   threadIdx.x, C_::kThreads);
   }
   // x rows M .. kXRows-1 of every stage are never copied: keep them zero (16-byte stores,
   // rows are 256 bytes)

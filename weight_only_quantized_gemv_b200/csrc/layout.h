@@ -57,7 +57,9 @@
 
 namespace qlayout {
 
-enum { kW2 = 2, kW3 = 3, kW4 = 4, kW8 = 8, kLUT4 = 16 };
+// kCB: a codebook of 256 fp16 4-vectors with 8-bit codes (m1v4g128) in the tensor-core GEMV
+// layout: per chunk lane, the code of each (step, row half) in one byte (2 s + r8)
+enum { kW2 = 2, kW3 = 3, kW4 = 4, kW8 = 8, kLUT4 = 16, kCB = 32 };
 
 constexpr int kGroup = 128;      // quantization group along K (uniform formats)
 constexpr int kLutBlock = 64;    // absmax block along K (LUT4)
@@ -66,7 +68,7 @@ constexpr int kBlockTiles = 8;   // tiles per block (128 columns)
 
 // 32-bit words of codes per lane per chunk.
 QL_HD int words_per_lane(int fmt) {
-  return fmt == kW2 ? 4 : fmt == kW3 ? 6 : fmt == kW8 ? 16 : 8;
+  return (fmt == kW2 || fmt == kCB) ? 4 : fmt == kW3 ? 6 : fmt == kW8 ? 16 : 8;
 }
 QL_HD int chunk_bytes(int fmt) { return 128 * words_per_lane(fmt); }
 QL_HD int code_bits(int fmt) { return fmt == kLUT4 ? 4 : fmt; }

@@ -127,6 +127,37 @@ extern "C" ql_status qlinear_pack_params(int fmt, const void* canonical, void* p
   return QL_OK;
 }
 
+// Codebook indices (canonical uint8 [K / 4][N]: the code of the 4-vector k = 4j .. 4j + 3 of
+// column n) into the tensor-core GEMV layout: chunks (block, group, tile) in the order of the
+// uniform formats, 512 bytes each, lane l's 16 bytes at 16 l; byte 2 s + r8 holds the code of
+// row 16 tile + gi + 8 r8 for step s, whose k are 128 g + k_in_group(s, t, 0 .. 3) (one whole
+// vector, since k_in_group(s, t, 0) is a multiple of 4).
+extern "C" ql_status qlinear_pack_codebook_tc(const uint8_t* codes, uint8_t* packed, int N, int K) {
+  if (!codes || !packed) return QL_ERR_NULL;
+  if (!shape_ok(N, K)) return QL_ERR_SHAPE;
+  const int G = K / kGroup;
+  const int ntiles = N / kTileN;
+  const int nblocks = (ntiles + kBlockTiles - 1) / kBlockTiles;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int b = 0; b < nblocks; ++b) {
+    const int tb = tiles_in_block(b, ntiles);
+    for (int g = 0; g < G; ++g)
+      for (int jj = 0; jj < tb; ++jj) {
+        uint8_t* chunk = packed + chunk_index(b, g, jj, G, ntiles) * 512;
+        const int n_base = (b * kBlockTiles + jj) * kTileN;
+        for (int lane = 0; lane < 32; ++lane) {
+          const int gi = lane >> 2, t = lane & 3;
+          for (int s = 0; s < 8; ++s)
+            for (int r8 = 0; r8 < 2; ++r8) {
+              const int j = (g * kGroup + k_in_group(s, t, 0)) / 4;
+              chunk[lane * 16 + 2 * s + r8] = codes[(size_t)j * N + n_base + gi + 8 * r8];
+            }
+        }
+      }
+  }
+  return QL_OK;
+}
+
 // Reorder Tile-COO tiles from the canonical K-major tile order (t = kt * NB + nt) to
 // the order the fused kernel walks them (t' = nt * (K / 128) + kt), so the outliers
 // of one run of work units are contiguous.  Entries keep their in-tile order.

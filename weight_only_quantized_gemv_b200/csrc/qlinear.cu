@@ -28,6 +28,8 @@ std::atomic<uint32_t> g_test_us{0};
 bool fmt_ok(int fmt) {
   return fmt == kW2 || fmt == kW3 || fmt == kW4 || fmt == kW8 || fmt == kLUT4;
 }
+// ... and the formats the GEMV (plan, workspace) also serves: the tensor-core codebook layout
+bool gemv_fmt_ok(int fmt) { return fmt_ok(fmt) || fmt == kCB; }
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -123,6 +125,7 @@ KernelInfo select_kernel(int fmt, int MT, bool outl, int wpu, bool m1, bool occ2
       if (MT == 2) return kernel_info<kW4, 2, false>();
       return wpu == 4 ? w4_m8_kernel<4>(m1) : wpu == 2 ? w4_m8_kernel<2>(m1) : w4_m8_kernel<1>(m1);
     case kW8: return MT == 1 ? m8_kernel<kW8, false>(m1) : kernel_info<kW8, 2, false>();
+    case kCB: return MT == 1 ? m8_kernel<kCB, false>(m1) : kernel_info<kCB, 2, false>();
     default: return MT == 1 ? m8_kernel<kLUT4, false>(m1) : kernel_info<kLUT4, 2, false>();
   }
 }
@@ -335,9 +338,12 @@ ql_status check_call(const Call& c) {
   if (!shape_ok(c.M, c.N, c.K)) return QL_ERR_SHAPE;
   if (c.outl && c.N % 128) return QL_ERR_SHAPE;
   if (!aligned(c.x, 16) || !aligned(c.qw, 32) || !aligned(c.y, 2)) return QL_ERR_ALIGN;
-  // parameters arrive by bulk copies (16-byte aligned sources); the LUT is read directly
+  // parameters arrive by bulk copies (16-byte aligned sources); the LUT and the codebook
+  // are read directly
   if (c.fmt == kLUT4) {
     if (!aligned(c.p0, 2) || !aligned(c.p1, 16)) return QL_ERR_ALIGN;
+  } else if (c.fmt == kCB) {
+    if (!aligned(c.p0, 16) || !aligned(c.p1, 8)) return QL_ERR_ALIGN;
   } else if (!aligned(c.p0, 16) || !aligned(c.p1, 16)) {
     return QL_ERR_ALIGN;
   }
@@ -531,11 +537,11 @@ extern "C" const char* ql_status_str(int status) {
 }
 
 extern "C" size_t qlinear_workspace_bytes(int fmt, int M, int N, int K) {
-  if (!fmt_ok(fmt) || !shape_ok(M, N, K)) return 0;
+  if (!gemv_fmt_ok(fmt) || !shape_ok(M, N, K)) return 0;
   Plan p;
   if (make_plan(fmt, M, N, K, false, &p) != cudaSuccess) return 0;
   // the finer-group kernels (group 64, 32) may resolve to another occupancy: cover them
-  if (fmt != kLUT4 && fmt != kW3) {
+  if (fmt != kLUT4 && fmt != kW3 && fmt != kCB) {
     for (int ns : {2, 4}) {
       Plan q;
       if (make_plan(fmt, M, N, K, false, &q, ns) == cudaSuccess && q.ws_bytes > p.ws_bytes)
@@ -552,7 +558,7 @@ extern "C" size_t qlinear_workspace_bytes(int fmt, int M, int N, int K) {
 
 extern "C" ql_status qlinear_plan(int fmt, int M, int N, int K, ql_plan* plan) {
   if (!plan) return QL_ERR_NULL;
-  if (!fmt_ok(fmt)) return QL_ERR_UNSUPPORTED;
+  if (!gemv_fmt_ok(fmt)) return QL_ERR_UNSUPPORTED;
   if (!shape_ok(M, N, K)) return QL_ERR_SHAPE;
   Plan p;
   if (make_plan(fmt, M, N, K, false, &p) != cudaSuccess) return QL_ERR_CUDA;
@@ -595,6 +601,15 @@ extern "C" ql_status qlinear_lut4(const uint16_t* x, const uint8_t* codes, const
                                   void* workspace, size_t workspace_bytes, ql_stream_t stream) {
   if (block != kLutBlock) return QL_ERR_SHAPE;
   Call c{kLUT4, false, x, codes, lut16, absmax, nullptr, nullptr, nullptr, y, M, N, K,
+         workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)};
+  return run(c);
+}
+
+extern "C" ql_status qlinear_codebook_tc(const uint16_t* x, const uint8_t* codes,
+                                         const uint16_t* scales, const uint16_t* codebook,
+                                         uint16_t* y, int M, int N, int K, void* workspace,
+                                         size_t workspace_bytes, ql_stream_t stream) {
+  Call c{kCB, false, x, codes, scales, codebook, nullptr, nullptr, nullptr, y, M, N, K,
          workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)};
   return run(c);
 }

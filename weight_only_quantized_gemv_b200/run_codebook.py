@@ -17,7 +17,8 @@ import math
 
 import torch
 
-from . import qlinear_codebook, qlinear_codebook_workspace_bytes
+from . import (QL_FMT_CB, qlinear_codebook, qlinear_codebook_tc, qlinear_codebook_workspace_bytes,
+                qlinear_workspace_bytes)
 
 L2_BYTES = 126 * 2 ** 20
 
@@ -33,6 +34,8 @@ def main() -> None:
     ap.add_argument("--M", type=int, default=1)
     ap.add_argument("--launches", type=int, default=30)
     ap.add_argument("--time", action="store_true")
+    ap.add_argument("--tc", action="store_true",
+                    help="the tensor-core form (qlinear_codebook_tc) instead of the Psumbook")
     a = ap.parse_args()
     K, N, M = a.K, a.N, a.M
     dev = torch.device("cuda:0")
@@ -47,12 +50,14 @@ def main() -> None:
     cb = (torch.rand(256 * 4, device=dev, generator=gen) * 2 - 1).half().view(torch.int16)
     x = torch.randn(M, K, device=dev, generator=gen).half().view(torch.int16)
     y = torch.empty(M, N, device=dev, dtype=torch.int16)
-    ws = torch.zeros(max(qlinear_codebook_workspace_bytes(M, N, K), 256) // 4 + 64,
-                     dtype=torch.int32, device=dev)
+    need = (qlinear_workspace_bytes(QL_FMT_CB, M, N, K) if a.tc
+            else qlinear_codebook_workspace_bytes(M, N, K))
+    ws = torch.zeros(max(need, 256) // 4 + 64, dtype=torch.int32, device=dev)
+    entry = qlinear_codebook_tc if a.tc else qlinear_codebook
 
     def call(i):
         c = i % copies
-        qlinear_codebook(x, codes[c], scales[c], cb, y, M, N, K, ws)
+        entry(x, codes[c], scales[c], cb, y, M, N, K, ws)
 
     if not a.time:
         for i in range(a.launches):
@@ -79,7 +84,7 @@ def main() -> None:
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / (reps * a.launches)
     b = algorithmic_bytes(K, N, M)
-    print(json.dumps({"fmt": "cb2", "K": K, "N": N, "M": M, "us": round(us, 3), "bytes": b,
+    print(json.dumps({"fmt": "cb2", "form": "tensor-core" if a.tc else "psumbook", "K": K, "N": N, "M": M, "us": round(us, 3), "bytes": b,
                       "GBs": round(b / us / 1e3, 1), "lookups": M * K * N // 4,
                       "Glookups_s": round(M * K * N / 4 / us / 1e3, 1)}))
 
