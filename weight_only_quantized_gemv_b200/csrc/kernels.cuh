@@ -108,7 +108,7 @@ template <> struct Fmt<kCB> {  // 8-bit codebook indices, two per step (rows gi,
   static constexpr int kWords = 4;
   static constexpr uint32_t kOnesHi = 0;
   static constexpr float kHiScale = 1.0f;
-  static constexpr int kStagesPerWarpM8 = 2;
+  static constexpr int kStagesPerWarpM8 = 1;  // with the 32 KB table: three CTAs per SM
 };
 template <> struct Fmt<kLUT4> {
   static constexpr int kWords = 8;
@@ -159,7 +159,7 @@ struct Cfg {
   // fewer registers per thread)
   static constexpr int kOcc = OCC_;
   static constexpr int kMinCtas =
-      OCC_ ? OCC_ : (FMT == kLUT4 || FMT == kCB) ? 2 : (MT == 1 && FMT != kW8) ? 3 : 2;
+      OCC_ ? OCC_ : (FMT == kLUT4) ? 2 : (MT == 1 && FMT != kW8) ? 3 : 2;
   static constexpr int kChunkBytes = 128 * KW;
   static constexpr int kCodeBytes = kBlockTiles * kChunkBytes;
   static constexpr int kParamChunk = (FMT == kLUT4) ? 128 : 32 * NS;   // per tile, per array
