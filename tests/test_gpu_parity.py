@@ -302,7 +302,10 @@ def test_workspace_too_small_is_rejected():
 def test_many_launches_bit_identical(kind, M):
     """A stage refilled before every lane has read it would show as results that differ
     between launches: 200 back-to-back launches on a layer whose CTAs each stream many units
-    (every ring wraps), all bit-identical to the first, the first within tolerance."""
+    (every ring wraps), all bit-identical to the first, the first within tolerance.  The
+    outlier kernel adds its outliers with shared-memory float atomics, whose order varies
+    between launches: there each launch must stay within tolerance and within one fp16
+    rounding of the first."""
     K, N = 4096, 2048
     x, xd = _x(773 + M, M, K)
     if kind == "lut4":
@@ -324,8 +327,15 @@ def test_many_launches_bit_identical(kind, M):
     torch.cuda.synchronize()
     first = y.view(torch.int16).cpu().numpy().copy()
     assert_parity(first.view(np.float16).astype(np.float64), want, what=f"{kind} M={M}")
+    f0 = first.view(np.float16).astype(np.float64)
     for _ in range(200):
         lay.forward(xd, y)
         torch.cuda.synchronize()
-        assert np.array_equal(y.view(torch.int16).cpu().numpy(), first)
+        h = y.view(torch.int16).cpu().numpy()
+        if kind != "outlier":
+            assert np.array_equal(h, first)
+        else:
+            f = h.view(np.float16).astype(np.float64)
+            assert np.all(np.abs(f - f0) <= 2.0 ** -10 * np.abs(f0) + 2.0 ** -24)
+            assert_parity(f, want, what=f"{kind} M={M}, repeated")
     assert lay.read_error() == 0
