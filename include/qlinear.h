@@ -76,7 +76,7 @@ typedef enum {
   QL_ERR_ALIGN = 3,       /* a pointer is not aligned as documented */
   QL_ERR_UNSUPPORTED = 4, /* unknown format */
   QL_ERR_WORKSPACE = 5,   /* workspace missing or smaller than qlinear_workspace_bytes() */
-  QL_ERR_CUDA = 6,        /* a CUDA runtime call, kernel launch or cuBLAS call failed */
+  QL_ERR_CUDA = 6,        /* a CUDA runtime call or kernel launch failed */
   QL_ERR_LIBRARY = 7      /* reserved (no library is opened at run time) */
 } ql_status;
 

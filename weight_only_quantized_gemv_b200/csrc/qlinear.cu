@@ -531,7 +531,7 @@ extern "C" const char* ql_status_str(int status) {
     case QL_ERR_UNSUPPORTED: return "unknown format";
     case QL_ERR_WORKSPACE: return "workspace missing or too small";
     case QL_ERR_CUDA: return "CUDA error";
-    case QL_ERR_LIBRARY: return "cuBLAS could not be loaded or initialised";
+    case QL_ERR_LIBRARY: return "reserved (no library is opened at run time)";
     default: return "unknown status";
   }
 }
