@@ -14,7 +14,7 @@
 //    and the last CTA to arrive at a block (atomic counter, no waiting) adds them
 //    up in a fixed order.
 //  * One producer warp streams the range through a ring of S shared-memory stages
-//    with non-multicast bulk copies (cp.async.bulk, TMA 1-D): per unit the codes of
+//    with plain bulk copies (cp.async.bulk, TMA 1-D, into its own CTA): per unit the codes of
 //    the block's tiles, their scales/zeros (or absmax) and the M rows of x for the
 //    group, all completing on the stage's mbarrier.  Weights and parameters carry
 //    an L2 evict-first hint: they are read once.  Bytes in flight are bounded by
