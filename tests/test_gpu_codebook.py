@@ -195,3 +195,17 @@ def test_tc_full_size_sampled(M):
     cols = np.unique(np.concatenate([rs.choice(L.N, 160, replace=False),
                                      [0, 15, 16, 127, 128, L.N - 129, L.N - 16, L.N - 1]]))
     assert_parity(y[:, cols], _ref(L, x, cols), what=f"cb tc full M={M}")
+
+
+@pytest.mark.parametrize("form,M", [("tc", 1), ("tc", 16), ("psumbook", 1), ("psumbook", 4)])
+def test_codebook_layer_both_forms(form, M):
+    """The device layer (layers.from_codebook) runs either form on the same canonical arrays."""
+    from weight_only_quantized_gemv_b200 import layers
+    K, N = 1024, 512
+    L = gen.codebook_layer(995, K, N)
+    lay = layers.from_codebook(L, DEV)
+    x = gen.activations(996 + M, M, K)
+    y = lay.forward(torch.from_numpy(x).to(DEV), form=form)
+    torch.cuda.synchronize()
+    assert lay.read_error() == 0
+    assert_parity(y.float().cpu().numpy(), _ref(L, x), what=f"cb layer {form} M={M}")

@@ -12,8 +12,10 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (QL_FMT_LUT4, QL_FMT_W2, QL_FMT_W3, QL_FMT_W4, QL_FMT_W8,
-               qlinear_debug_dequant,
+from . import (QL_FMT_CB, QL_FMT_LUT4, QL_FMT_W2, QL_FMT_W3, QL_FMT_W4, QL_FMT_W8,
+               qlinear_codebook, qlinear_codebook_tc, qlinear_codebook_workspace_bytes,
+               qlinear_debug_dequant, qlinear_pack_codebook, qlinear_pack_codebook_scales,
+               qlinear_pack_codebook_tc,
                qlinear_debug_unpack, qlinear_dequant_fp16, qlinear_lut4, qlinear_pack,
                qlinear_matmul, qlinear_pack_params, qlinear_pack_params_grouped,
                qlinear_prefill, qlinear_prefill_fused, qlinear_prefill_workspace_bytes,
@@ -195,3 +197,58 @@ def from_outlier(layer, device="cuda", max_m: int = 16) -> QuantLinear:
     return QuantLinear(QL_FMT_W4, d.K, d.N, d.qweight, d.scales, d.zeros,
                        tilecoo=(layer.tile_offsets, layer.tile_rc, layer.tile_vals),
                        device=device, max_m=max_m)
+
+
+class CodebookLinear:
+    """A codebook-quantized weight matrix (m1v4g128: codes uint8 [K / 4][N], scales fp16
+    [K / 128][N], codebook fp16 [256][4]) on the device, packed for both GEMV forms: the
+    Psumbook form (``qlinear_codebook``, M <= 4, N % 32 == 0) and the tensor-core form
+    (``qlinear_codebook_tc``, M <= 16, N % 16 == 0)."""
+
+    def __init__(self, K: int, N: int, codes: np.ndarray, scales: np.ndarray,
+                 codebook: np.ndarray, device="cuda", max_m: int = 16):
+        self.K, self.N, self.device, self.max_m = K, N, torch.device(device), max_m
+        scales16 = np.ascontiguousarray(scales).view(np.uint16)
+        self.codebook = _dev(np.ascontiguousarray(codebook).view(np.int16), self.device)
+        self.codes_tc = _dev(qlinear_pack_codebook_tc(codes, N, K), self.device)
+        self.scales_tc = _dev(qlinear_pack_params(QL_FMT_W4, scales16, N, K).view(np.int16),
+                              self.device)
+        ws = max(qlinear_workspace_bytes(QL_FMT_CB, m, N, K) for m in (1, max_m))
+        self.ws_tc = torch.zeros(max(ws, 256) // 4 + 64, dtype=torch.int32, device=self.device)
+        self.psum_ok = N % 32 == 0
+        if self.psum_ok:
+            self.codes_ps = _dev(qlinear_pack_codebook(codes, N, K), self.device)
+            self.scales_ps = _dev(qlinear_pack_codebook_scales(scales16, N, K).view(np.int16),
+                                  self.device)
+            ws = max(qlinear_codebook_workspace_bytes(m, N, K) for m in range(1, 5))
+            self.ws_ps = torch.zeros(max(ws, 256) // 4 + 64, dtype=torch.int32,
+                                     device=self.device)
+
+    def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, stream=None,
+                form: str = "tc") -> torch.Tensor:
+        """y[M, N] (fp16) = x[M, K] (fp16) . W; form "tc" (tensor cores) or "psumbook"."""
+        M = x.shape[0]
+        if y is None:
+            y = torch.empty((M, self.N), dtype=torch.float16, device=self.device)
+        xv, yv = x.view(torch.int16), y.view(torch.int16)
+        if form == "tc":
+            qlinear_codebook_tc(xv, self.codes_tc, self.scales_tc, self.codebook, yv, M, self.N,
+                                self.K, self.ws_tc, stream)
+        elif form == "psumbook":
+            if not self.psum_ok:
+                raise ValueError("the Psumbook form needs N % 32 == 0")
+            qlinear_codebook(xv, self.codes_ps, self.scales_ps, self.codebook, yv, M, self.N,
+                             self.K, self.ws_ps, stream)
+        else:
+            raise ValueError(f"unknown form {form!r}")
+        return y
+
+    def read_error(self, stream=None) -> int:
+        """Sticky error flags of the tensor-core form's device waits (then cleared)."""
+        return qlinear_read_error(self.ws_tc, stream)
+
+
+def from_codebook(layer, device="cuda", max_m: int = 16) -> CodebookLinear:
+    """From a ``synth.gen.CodebookLayer``-like object (K, N, codes, scales, codebook)."""
+    return CodebookLinear(layer.K, layer.N, layer.codes, layer.scales, layer.codebook,
+                          device=device, max_m=max_m)
