@@ -6,31 +6,35 @@
 // For M >> 16 the layer is compute-bound (QFactory page, assumption stress test and
 // limitation 1), and the weights are dequantized once per tile instead of once per 16 rows
 // of x.  Two forms of the A operand (the weights):
-//  * FUSED: producer warps read the packed codes and their scales / zeros (absmax) from
-//    global memory, dequantize them in registers to the same fp16 values the stand-alone
-//    dequantization writes ("Fast NF4 Dequantization Kernels" page, method section: codes
-//    -> FP16 -> matmul; here FP16 goes to shared memory instead of back to HBM), and store
-//    them into the shared-memory operand of the MMAs;
+//  * FUSED: dequantizing warps decode the packed codes and their scales / zeros (absmax),
+//    which a producer warp brings into shared memory by TMA, to the same fp16 values the
+//    stand-alone dequantization writes ("Fast NF4 Dequantization Kernels" page, method
+//    section: codes -> FP16 -> matmul; here FP16 goes to shared memory instead of back to
+//    HBM), and store them into the shared-memory operand of the MMAs;
 //  * dense: a TMA tensor copy of an fp16 W[N][K] (the stand-alone dequantization's output).
 //
 // Design:
-//  * One persistent CTA per SM; output tiles of 128 weight rows (the MMA's M: output
-//    columns n) x BN rows of x (the MMA's N: tokens), taken in turn by the CTAs.
-//  * A ring of S shared-memory stages of 64 k each: A 128 x 64 and B BN x 64 fp16, both in
-//    the K-major 128-byte-swizzled layout (rows of 128 bytes, 16-byte granule c of row r at
-//    granule c ^ (r mod 8)), which is what the TMA copy with 128-byte swizzle writes.
+//  * One persistent CTA per SM (or cluster pair of CTAs on two SMs: tcgen05 cta_group::2,
+//    256-row tiles); output tiles of 128 weight rows per CTA (the MMA's M: output columns n)
+//    x BN rows of x (the MMA's N: tokens), taken in turn by the CTAs, or shared out by
+//    k-block with a workspace (stream-K).
+//  * A ring of S shared-memory stages of 64 k each: A 128 x 64 and B (BN / CTAs) x 64 fp16,
+//    both in the K-major 128-byte-swizzled layout (rows of 128 bytes, 16-byte granule c of
+//    row r at granule c ^ (r mod 8)), which is what the TMA copy with 128-byte swizzle
+//    writes.  FUSED: the codes in a ring of their own, filled ahead of the stages.
 //  * Warp 0: one lane issues the TMA copies (x, and W in the dense form).  Warp 1: one lane
-//    issues tcgen05.mma (M = 128, N = BN, K = 16; four per stage) and tcgen05.commit, which
-//    releases a stage once the MMAs that read it are done; the warp owns the tensor memory.
-//    Warps 2..5: epilogue (tcgen05.ld of the accumulator, fp16 stores).  FUSED: warps
-//    6..13 dequantize (one 16-column tile of the 128 rows each).
+//    issues tcgen05.mma (K = 16; four per stage) and tcgen05.commit, which releases a stage
+//    once the MMAs that read it are done; the warp owns the tensor memory.  Warps 2..5:
+//    epilogue (tcgen05.ld of the accumulator, fp16 stores).  FUSED: warps 6..13 dequantize
+//    (one 16-column tile of the 128 rows each), warp 14 copies the codes.
 //  * Two accumulators of BN fp32 columns in tensor memory: the epilogue of one tile
 //    overlaps the MMAs of the next.
-//  * Every mbarrier wait is bounded in time (100 ms; a healthy one takes microseconds).  One
-//    that runs out sets a flag in a device error word (qlinear_prefill_read_error) and a
-//    CTA-wide abort flag; every role then leaves its loop, waits briefly for its copies and
-//    MMAs in flight, and the CTA releases its tensor memory and exits.  A lost copy gives
-//    wrong numbers, never a hung GPU.
+//  * Every mbarrier wait first tests the phase inline; one that has to wait is bounded in
+//    time (100 ms; a healthy one takes microseconds).  One that runs out sets a flag in a
+//    device error word (qlinear_prefill_read_error) and a CTA-wide abort flag; every role
+//    then leaves its loop, waits briefly for its copies and MMAs in flight, and the CTA
+//    releases its tensor memory and exits.  A lost copy gives wrong numbers, never a hung
+//    GPU.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
