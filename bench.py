@@ -120,6 +120,15 @@ def generate_all(specs, procs):
     return dict(zip(order, layers))
 
 
+def replay_plan(n):
+    """Graph sizes (steps per replay) that run exactly n steps: a one-step graph first (it
+    launches fastest, so the device starts almost at once while the host enqueues the rest),
+    then ten-step graphs, then one-step graphs for the remainder."""
+    if n <= 0:
+        return []
+    return [1] + [10] * ((n - 1) // 10) + [1] * ((n - 1) % 10)
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
@@ -531,15 +540,8 @@ def run_gpu(args):
     torch.cuda.synchronize()
 
     def steps(n):
-        # a one-step graph first: it launches fastest, so the device starts almost at once
-        # while the host enqueues the ten-step graphs behind it
-        if n <= 0:
-            return
-        g1.replay()
-        for _ in range((n - 1) // 10):
-            g10.replay()
-        for _ in range((n - 1) % 10):
-            g1.replay()
+        for size in replay_plan(n):
+            (g10 if size == 10 else g1).replay()
 
     # The other measurements run before the timed region: they bring the GPU from idle to
     # its steady clocks and power state, which a short timed region (a few ms) would

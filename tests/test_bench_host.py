@@ -62,3 +62,15 @@ def test_oracle_timing_counts_sample_bytes():
     # the bytes of one call: 16 columns' codes and parameters, x (2 rows) and 16 y columns
     per_call = bench.format_bytes("w4", 256, 16, 2)
     assert gbs == pytest.approx(calls * per_call / secs / 1e9, rel=1e-9)
+
+
+def test_replay_plan_runs_exactly_n_steps():
+    """The timed region replays graphs of 10 and 1 steps; the plan must add up to exactly the
+    requested steps, start with the one-step graph and use few replays."""
+    for n in range(0, 200):
+        plan = bench.replay_plan(n)
+        assert sum(plan) == n
+        assert set(plan) <= {1, 10}
+        if n:
+            assert plan[0] == 1
+            assert len(plan) <= 1 + n // 10 + 9
